@@ -1,0 +1,175 @@
+/*
+ * moe.h - C ABI of libmoe.so: one block-quantized, top-k routed Mixture-of-
+ * Experts FFN layer on an NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources: the "Strata Coder deep-dive" page, sections 1-3, and the
+ * "Coder benchmark record" page, "why Coder is fast" and "expert profile file"
+ * sections):
+ *   - each token of hidden size H is routed to top_k of the E experts of a
+ *     layer (48 layers x 512 experts, or 256 after pruning; top_k = 10);
+ *   - an expert is three block-quantized projections, gate and up [I, H] and
+ *     down [H, I], each with its own bit width (2 or 4), held in an expert
+ *     arena addressed per (layer, expert);
+ *   - routing counts per (layer, expert) accumulate into a histogram whose
+ *     ranking is the expert profile.
+ * Computation, per token t:
+ *   l_e   = x_t . W_r[e] + b_e                      (router logits)
+ *   S_t   = the top_k experts by (l desc, e asc)    (bit-exact vs fp64 math)
+ *   w_j   = softmax over the chosen logits
+ *   y_e   = W_d (silu(W_g x_t) * (W_u x_t))         (SwiGLU expert)
+ *   out_t = (residual ? x_t : 0) + sum_j w_j y_{S_t[j]}   rounded to bf16.
+ * Dequantised weight: scale_fp16[row][c/32] * (code - 2^(bits-1)).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked (device) are caller-owned device memory, (host) are
+ *     host memory.  The library allocates nothing on any call path.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device work
+ *     is enqueued asynchronously on it; the call returns once it is enqueued.
+ *   - Return value: MOE_OK or a negative MOE_ERR_* code.  Errors found on the
+ *     host (arguments, shapes, workspace) launch nothing.  Errors found on the
+ *     device (a selected expert without a valid slot, a bounded wait that
+ *     expired) are latched in a per-device status word read by
+ *     moe_last_device_error().
+ *   - x and out must not overlap.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_ARG (-1)      /* null or misaligned pointer, overlapping x/out  */
+#define MOE_ERR_SHAPE (-2)    /* H, I, block or bit widths not supported        */
+#define MOE_ERR_RANGE (-3)    /* T, E, top_k or layer outside its bound         */
+#define MOE_ERR_WS (-4)       /* workspace smaller than moe_workspace_bytes()   */
+#define MOE_ERR_CUDA (-5)     /* a CUDA launch or query failed                  */
+#define MOE_ERR_SLOT (-6)     /* a selected expert had slot -1 or >= n_slots    */
+#define MOE_ERR_TIMEOUT (-7)  /* a bounded device-side wait expired             */
+
+#define MOE_MAX_E 512         /* experts per layer                              */
+#define MOE_MAX_TOPK 32
+#define MOE_DECODE_MAX_T 8    /* decode path: a verify window of 1 + 4 drafts fits */
+#define MOE_PREFILL_MAX_T 8192 /* one prefill chunk                             */
+
+/*
+ * Expert-slot layout, identical for every slot of an arena.  Matrix m is
+ * 0 = gate [I, H], 1 = up [I, H], 2 = down [H, I], row-major by output row;
+ * quant blocks of `block` (= 32) elements run along the reduction axis.
+ * Codes: row r of a b-bit matrix with reduction length K occupies K*b/8
+ * bytes at off_codes[m] + r*K*b/8; element c sits at byte c*b/8 of the row,
+ * bit offset (c*b) % 8, least significant bits first.  Scales: fp16
+ * [rows][K/32] at off_scales[m].  Slot s starts at arena + s*slot_bytes.
+ * Requirements (else MOE_ERR_SHAPE): block == 32, H % 32 == 0, I % 32 == 0,
+ * 32 <= H <= 8192, 32 <= I <= 4096, bits in {2, 4}, slot_bytes % 256 == 0,
+ * every offset % 128 == 0 with its section inside the slot, n_slots >= 1,
+ * reserved == 0.  The prefill path also needs H % 128 == 0 and I % 128 == 0.
+ */
+typedef struct moe_arena_desc {
+    int32_t H, I, block;
+    int32_t bits_gate, bits_up, bits_down;
+    int64_t slot_bytes;
+    int64_t off_codes[3];
+    int64_t off_scales[3];
+    int32_t n_slots;
+    int32_t reserved;        /* must be 0 */
+} moe_arena_desc;
+
+/*
+ * Optional routing outputs of a forward call.  Each non-NULL pointer is a
+ * device buffer the call fills (it is also used as the working copy, so
+ * passing it costs no extra traffic):
+ *   topk_idx [T*top_k] int32  experts of token t in slots j = 0..k-1,
+ *                             ordered by logit desc, ties by lower index
+ *   topk_w   [T*top_k] fp32   gate weights (softmax over the k chosen logits)
+ *   expert_offsets [E+1]      exclusive prefix sum of per-expert pair counts
+ *   perm     [T*top_k] int32  pair ids p = t*k + j grouped by expert,
+ *                             ascending p inside an expert
+ *   n_rechecked [1] int32     tokens whose selection needed the exact fp64
+ *                             re-evaluation (diagnostic)
+ */
+typedef struct moe_route_out {
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* expert_offsets;
+    int32_t* perm;
+    int32_t* n_rechecked;
+} moe_route_out;
+
+/* Bytes of scratch workspace a forward (or moe_route) call with these sizes
+ * needs; pass it as `ws` (device, 256-byte aligned).  Host only, no CUDA. */
+size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I);
+
+/*
+ * Router and grouping only.
+ *   x [T][H] bf16 (device, 16-B aligned), router_w [E][H] fp32 (device,
+ *   16-B aligned), router_bias [E] fp32 (device) or NULL.
+ *   Outputs (device): topk_idx [T*k], topk_w [T*k], expert_offsets [E+1],
+ *   perm [T*k].  1 <= T <= 8192, 1 <= E <= 512, 1 <= top_k <= min(E, 32).
+ *   T = 0 is a no-op returning MOE_OK.
+ */
+int moe_route(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias,
+              int E, int top_k, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+              int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Full layer for a decode window, 1 <= T <= MOE_DECODE_MAX_T: router, grouping,
+ * fused dequant + SwiGLU gate/up, down projection, weighted combine (+x when
+ * residual != 0) and, when hist != NULL, hist[layer][e] += pairs routed to e.
+ *   desc (host); arena (device, 256-B aligned); slot_table [L][E] int32
+ *   (device); x [T][H] bf16 (device); out [T][H] bf16 (device);
+ *   hist [L][E] uint32 (device, persistent, caller-owned) or NULL;
+ *   route_out (host struct of device pointers) or NULL.
+ *   0 <= layer < L.  T = 0 is a no-op.
+ */
+int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
+                       int L, int layer, const uint16_t* x, int T, const float* router_w,
+                       const float* router_bias, int E, int top_k, int residual, uint16_t* out,
+                       uint32_t* hist, const moe_route_out* route_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Full layer for a prefill chunk, 1 <= T <= MOE_PREFILL_MAX_T: same arguments
+ * and results as moe_forward_decode; the expert FFN runs as per-expert grouped
+ * GEMMs on the tensor cores (weights dequantised to bf16 on chip, SwiGLU
+ * output h rounded to bf16, per-pair expert outputs kept in bf16).
+ */
+int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
+                        int L, int layer, const uint16_t* x, int T, const float* router_w,
+                        const float* router_bias, int E, int top_k, int residual, uint16_t* out,
+                        uint32_t* hist, const moe_route_out* route_out, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * Routing-count histogram ("--dump-routing" counts of the benchmark record
+ * page): hist[layer][e] += expert_offsets[e+1] - expert_offsets[e] for
+ * e < E, one owner thread per expert, no atomics.  expert_offsets [E+1]
+ * (device), hist [L][E] uint32 (device).
+ */
+int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, uint32_t* hist,
+                        void* stream);
+
+/*
+ * Expert-profile ranking (Strata Coder deep-dive page, section 3; benchmark
+ * record page, "expert profile file"): every (layer, expert) pair ordered by
+ * count descending, ties by (layer, expert) ascending.
+ *   hist_host [L][E] uint32 (host); pairs_out [L*E][2] uint16 (host) =
+ *   (layer, expert) of rank 0, 1, ...  Host only, no CUDA.
+ */
+int moe_rank_experts(const uint32_t* hist_host, int L, int E, uint16_t* pairs_out);
+
+/* Reads and clears the current device's status word after synchronising
+ * `stream`: MOE_OK, MOE_ERR_SLOT or MOE_ERR_TIMEOUT (the first latched). */
+int moe_last_device_error(void* stream);
+
+/* Static message for a return code. */
+const char* moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -1,0 +1,417 @@
+// libmoe.so: the C ABI declared in include/moe.h.  Host code validates every
+// argument before the first CUDA call, lays out the caller's workspace, encodes
+// TMA descriptors and enqueues the kernels of router.cuh, perm.cuh, decode.cuh
+// and prefill.cuh on the caller's stream.  Nothing here allocates memory.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "perm.cuh"
+#include "prefill.cuh"
+#include "router.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Ws {
+    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, total;
+};
+
+inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
+
+Ws ws_layout(int T, int E, int k, int H, int I) {
+    const size_t P = (size_t)T * k;
+    const size_t nch = (P + PERM_CHUNK - 1) / PERM_CHUNK;
+    const bool small = T <= MOE_DECODE_MAX_T;
+    Ws w{};
+    size_t o = 0;
+    auto put = [&](size_t bytes) { size_t r = o; o += al(std::max<size_t>(bytes, 1)); return r; };
+    w.idx = put(P * 4);
+    w.w = put(P * 4);
+    w.logit = put((size_t)T * E * 4);
+    w.absum = put(small ? (size_t)T * E * 4 : 0);
+    w.cmax = put((size_t)(H + 1) * 4);
+    w.offsets = put((size_t)(E + 1) * 4);
+    w.perm = put(P * 4);
+    w.inv = put(P * 4);
+    w.uniq = put((size_t)E * 4);
+    w.meta = put(16);
+    w.chunk = put(nch * E * 4);
+    w.tiles = put((size_t)max_tiles((int)P, E) * 16);
+    w.nrechk = put(4);
+    w.xp = put(P * H * 2);
+    w.h = put(P * I * (small ? 4 : 2));  // decode keeps h and Y in fp32, prefill in bf16
+    w.y = put(P * H * (small ? 4 : 2));
+    w.total = o;
+    return w;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_desc(const moe_arena_desc* d, bool prefill) {
+    if (!d) return MOE_ERR_ARG;
+    if (d->block != 32 || d->reserved != 0) return MOE_ERR_SHAPE;
+    if (d->H < 32 || d->H > 8192 || d->H % 32 || d->I < 32 || d->I > 4096 || d->I % 32) return MOE_ERR_SHAPE;
+    if (prefill && (d->H % 128 || d->I % 128)) return MOE_ERR_SHAPE;
+    const int bits[3] = {d->bits_gate, d->bits_up, d->bits_down};
+    if (d->slot_bytes <= 0 || d->slot_bytes % 256 || d->n_slots < 1) return MOE_ERR_SHAPE;
+    for (int m = 0; m < 3; ++m) {
+        if (bits[m] != 2 && bits[m] != 4) return MOE_ERR_SHAPE;
+        const int64_t rows = m < 2 ? d->I : d->H, K = m < 2 ? d->H : d->I;
+        const int64_t cb = rows * K * bits[m] / 8, sb = rows * (K / 32) * 2;
+        if (d->off_codes[m] < 0 || d->off_codes[m] % 128 || d->off_codes[m] + cb > d->slot_bytes) return MOE_ERR_SHAPE;
+        if (d->off_scales[m] < 0 || d->off_scales[m] % 128 || d->off_scales[m] + sb > d->slot_bytes)
+            return MOE_ERR_SHAPE;
+    }
+    return MOE_OK;
+}
+
+int check_route_args(const uint16_t* x, int T, int H, const float* W, int E, int k, const void* ws, int maxT) {
+    if (T < 0 || T > maxT) return MOE_ERR_RANGE;
+    if (E < 1 || E > MOE_MAX_E || k < 1 || k > std::min(E, MOE_MAX_TOPK)) return MOE_ERR_RANGE;
+    if (H < 32 || H > 8192 || H % 32) return MOE_ERR_SHAPE;
+    if (!x || !W || !ws) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(W, 16) || !aligned(ws, kAlign)) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+inline float gamma32(int n) {
+    const double nu = (double)n * 5.9604644775390625e-8;  // n * 2^-24
+    return (float)(nu / (1.0 - nu));
+}
+
+inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Router + grouping on the caller's stream.  idx/w/offsets/perm may be the
+// caller's buffers or workspace.
+int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b, int E, int k, int32_t* idx,
+                 float* w, int32_t* offsets, int32_t* perm, int32_t* nrechk, uint8_t* ws, const Ws& L, bool want_tiles,
+                 uint32_t* hist, int layer, cudaStream_t st) {
+    const int P = T * k;
+    float* logit = reinterpret_cast<float*>(ws + L.logit);
+    int32_t* nr = nrechk ? nrechk : reinterpret_cast<int32_t*>(ws + L.nrechk);
+    if (cudaMemsetAsync(nr, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    TopkArgs ta{};
+    ta.x = x; ta.W = W; ta.b = b; ta.logit = logit; ta.idx = idx; ta.w = w; ta.n_rechecked = nr;
+    ta.T = T; ta.H = H; ta.E = E; ta.k = k;
+    if (T <= MOE_DECODE_MAX_T) {
+        float* absum = reinterpret_cast<float*>(ws + L.absum);
+        k_router_gemv<<<(E + 7) / 8, 256, 0, st>>>(x, T, H, W, b, E, logit, absum);
+        ta.absum = absum;
+        ta.gamma32 = gamma32(H / 32 + 6);
+    } else {
+        unsigned int* cmax = reinterpret_cast<unsigned int*>(ws + L.cmax);
+        if (cudaMemsetAsync(cmax, 0, (size_t)(H + 1) * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+        k_router_colmax<<<dim3((H + 1 + 255) / 256, (E + 31) / 32), 256, 0, st>>>(W, b, E, H, cmax);
+        k_router_gemm<<<dim3((E + RG_BN - 1) / RG_BN, (T + RG_BM - 1) / RG_BM), 256, 0, st>>>(x, T, H, W, b, E, logit);
+        ta.absum = nullptr;
+        ta.cmax = cmax;
+        ta.gamma32 = gamma32(H + 2);
+    }
+    k_topk<<<(T + MOE_TOPK_WARPS - 1) / MOE_TOPK_WARPS, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+    PermArgs pa{};
+    pa.idx = idx; pa.P = P; pa.E = E; pa.nchunks = (P + PERM_CHUNK - 1) / PERM_CHUNK;
+    pa.chunk_cnt = reinterpret_cast<int32_t*>(ws + L.chunk);
+    pa.offsets = offsets; pa.perm = perm;
+    pa.inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    pa.uniq = reinterpret_cast<int32_t*>(ws + L.uniq);
+    pa.meta = reinterpret_cast<int32_t*>(ws + L.meta);
+    pa.tiles = want_tiles ? reinterpret_cast<int4*>(ws + L.tiles) : nullptr;
+    pa.hist = hist; pa.layer = layer;
+    k_perm_count<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
+    k_perm_scan<<<1, MOE_MAX_E, 0, st>>>(pa);
+    k_perm_scatter<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
+    return cuda_rc(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode;
+}
+
+// bf16 [rows][K] row-major, box 64 x PF_BOX_ROWS, 128-byte swizzle
+bool tmap_act(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {PF_BK, PF_BOX_ROWS};
+    cuuint32_t es[2] = {1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// codes of one matrix across all slots: uint8 [n_slots][rows][row_bytes], box (PF_BK*bits/8) x 128 x 1
+bool tmap_codes(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t n_slots,
+                int64_t slot_bytes, int bits) {
+    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_slots};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)slot_bytes};
+    cuuint32_t box[3] = {(cuuint32_t)(PF_BK * bits / 8), PF_BM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- decode / prefill drivers
+
+namespace {
+
+struct LayerCall {
+    const moe_arena_desc* d;
+    const uint8_t* arena;
+    const int32_t* slot_table;
+    int L, layer;
+    const uint16_t* x;
+    int T;
+    const float* W;
+    const float* b;
+    int E, k, residual;
+    uint16_t* out;
+    uint32_t* hist;
+    const moe_route_out* ro;
+    uint8_t* ws;
+    size_t ws_bytes;
+    cudaStream_t st;
+};
+
+int check_layer(const LayerCall& c, bool prefill) {
+    int rc = check_desc(c.d, prefill);
+    if (rc) return rc;
+    rc = check_route_args(c.x, c.T, c.d->H, c.W, c.E, c.k, c.ws, prefill ? MOE_PREFILL_MAX_T : MOE_DECODE_MAX_T);
+    if (rc) return rc;
+    if (c.L < 1 || c.layer < 0 || c.layer >= c.L) return MOE_ERR_RANGE;
+    if (!c.arena || !c.slot_table || !c.out) return MOE_ERR_ARG;
+    if (!aligned(c.arena, 256) || !aligned(c.out, 16)) return MOE_ERR_ARG;
+    const size_t xb = (size_t)c.T * c.d->H * 2;
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(c.x), o0 = reinterpret_cast<uintptr_t>(c.out);
+    if (c.T > 0 && x0 < o0 + xb && o0 < x0 + xb) return MOE_ERR_ARG;
+    if (c.ws_bytes < ws_layout(c.T, c.E, c.k, c.d->H, c.d->I).total) return MOE_ERR_WS;
+    return MOE_OK;
+}
+
+struct Routed {
+    int32_t *idx, *offsets, *perm;
+    float* w;
+};
+
+int route_for_layer(const LayerCall& c, const Ws& L, bool tiles, Routed& r) {
+    const moe_route_out* ro = c.ro;
+    r.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
+    r.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
+    r.offsets = (ro && ro->expert_offsets) ? ro->expert_offsets : reinterpret_cast<int32_t*>(c.ws + L.offsets);
+    r.perm = (ro && ro->perm) ? ro->perm : reinterpret_cast<int32_t*>(c.ws + L.perm);
+    return launch_route(c.x, c.T, c.d->H, c.W, c.b, c.E, c.k, r.idx, r.w, r.offsets, r.perm,
+                        ro ? ro->n_rechecked : nullptr, c.ws, L, tiles, c.hist, c.layer, c.st);
+}
+
+template <int BG, int BU>
+void launch_gateup(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
+    const int smem = T * a.H * 2;
+    set_smem(k_dec_gateup<BG, BU>, smem);
+    k_dec_gateup<BG, BU><<<dim3((a.I + 31) / 32, umax), 32 * DEC_GU_WARPS, smem, st>>>(a);
+}
+
+template <int BD>
+void launch_down(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
+    const int smem = T * a.I * 4;
+    set_smem(k_dec_down<BD>, smem);
+    k_dec_down<BD><<<dim3((a.H + 31) / 32, umax), 32 * DEC_DN_WARPS, smem, st>>>(a);
+}
+
+int run_decode(const LayerCall& c) {
+    const moe_arena_desc* d = c.d;
+    const Ws L = ws_layout(c.T, c.E, c.k, d->H, d->I);
+    Routed r;
+    int rc = route_for_layer(c, L, false, r);
+    if (rc) return rc;
+    DecodeArgs a{};
+    a.arena = c.arena; a.slot_table = c.slot_table; a.slot_bytes = d->slot_bytes; a.n_slots = d->n_slots;
+    for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
+    a.H = d->H; a.I = d->I; a.E = c.E; a.k = c.k; a.layer = c.layer;
+    a.x = c.x; a.offsets = r.offsets; a.perm = r.perm;
+    a.uniq = reinterpret_cast<int32_t*>(c.ws + L.uniq);
+    a.meta = reinterpret_cast<int32_t*>(c.ws + L.meta);
+    a.topk_w = r.w;
+    a.h = reinterpret_cast<float*>(c.ws + L.h);
+    a.y = reinterpret_cast<float*>(c.ws + L.y);
+    const int umax = std::min(c.E, c.T * c.k);
+    if (d->bits_gate == 4 && d->bits_up == 4) launch_gateup<4, 4>(a, umax, c.T, c.st);
+    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gateup<2, 2>(a, umax, c.T, c.st);
+    else if (d->bits_gate == 2) launch_gateup<2, 4>(a, umax, c.T, c.st);
+    else launch_gateup<4, 2>(a, umax, c.T, c.st);
+    if (d->bits_down == 4) launch_down<4>(a, umax, c.T, c.st);
+    else launch_down<2>(a, umax, c.T, c.st);
+    k_combine<float><<<dim3((d->H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+        c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, d->H, c.k, c.residual, c.out);
+    return cuda_rc(cudaGetLastError());
+}
+
+template <int MODE, int B0, int B1>
+void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, const PrefillArgs& a,
+                 int mtiles, int ntile_max, cudaStream_t st) {
+    set_smem(k_prefill_gemm<MODE, B0, B1>, PfCfg<MODE>::SMEM);
+    k_prefill_gemm<MODE, B0, B1><<<dim3(mtiles, ntile_max), PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
+}
+
+int run_prefill(const LayerCall& c) {
+    const moe_arena_desc* d = c.d;
+    const int H = d->H, I = d->I, P = c.T * c.k;
+    const Ws L = ws_layout(c.T, c.E, c.k, H, I);
+    if (!encoder()) return MOE_ERR_CUDA;
+    Routed r;
+    int rc = route_for_layer(c, L, true, r);
+    if (rc) return rc;
+    uint16_t* xp = reinterpret_cast<uint16_t*>(c.ws + L.xp);
+    uint16_t* h = reinterpret_cast<uint16_t*>(c.ws + L.h);
+    uint16_t* y = reinterpret_cast<uint16_t*>(c.ws + L.y);
+    k_gather_rows<<<P, 128, 0, c.st>>>(c.x, r.perm, P, H, c.k, xp);
+    CUtensorMap tx, th, tg, tu, tdn;
+    const int64_t ns = d->n_slots, sb = d->slot_bytes;
+    if (!tmap_act(&tx, xp, P, H) || !tmap_act(&th, h, P, I) ||
+        !tmap_codes(&tg, c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8, ns, sb, d->bits_gate) ||
+        !tmap_codes(&tu, c.arena + d->off_codes[1], I, (int64_t)H * d->bits_up / 8, ns, sb, d->bits_up) ||
+        !tmap_codes(&tdn, c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb, d->bits_down))
+        return MOE_ERR_CUDA;
+    PrefillArgs a{};
+    a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = ns; a.slot_bytes = sb;
+    for (int m = 0; m < 3; ++m) a.off_scales[m] = d->off_scales[m];
+    a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer;
+    a.tiles = reinterpret_cast<const int4*>(c.ws + L.tiles);
+    a.meta = reinterpret_cast<const int32_t*>(c.ws + L.meta);
+    a.perm = r.perm; a.topk_w = r.w;
+    const int nt = max_tiles(P, c.E);
+    a.out = h;
+    if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    else launch_gemm<0, 4, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    a.out = y;
+    if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
+    else launch_gemm<1, 2, 2>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
+    k_combine<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+        c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);
+    return cuda_rc(cudaGetLastError());
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- exported entry points
+
+extern "C" {
+
+size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I) {
+    if (T < 0 || E < 1 || top_k < 1 || H < 1 || I < 1) return 0;
+    return ws_layout(T, E, top_k, H, I).total;
+}
+
+int moe_route(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias, int E, int top_k,
+              int32_t* topk_idx, float* topk_w, int32_t* expert_offsets, int32_t* perm, void* ws, size_t ws_bytes,
+              void* stream) {
+    int rc = check_route_args(x, T, H, router_w, E, top_k, ws, MOE_PREFILL_MAX_T);
+    if (rc) return rc;
+    if (!topk_idx || !topk_w || !expert_offsets || !perm) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    const Ws L = ws_layout(T, E, top_k, H, 32);
+    if (ws_bytes < L.total) return MOE_ERR_WS;
+    return launch_route(x, T, H, router_w, router_bias, E, top_k, topk_idx, topk_w, expert_offsets, perm, nullptr,
+                        static_cast<uint8_t*>(ws), L, false, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L,
+                   int layer, const uint16_t* x, int T, const float* router_w, const float* router_bias, int E,
+                   int top_k, int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                   size_t ws_bytes, void* stream) {
+    LayerCall c{desc, static_cast<const uint8_t*>(arena), slot_table, L, layer, x, T, router_w, router_bias, E,
+                top_k, residual, out, hist, route_out, static_cast<uint8_t*>(ws), ws_bytes,
+                static_cast<cudaStream_t>(stream)};
+    int rc = check_layer(c, prefill);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    return prefill ? run_prefill(c) : run_decode(c);
+}
+
+int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L, int layer,
+                       const uint16_t* x, int T, const float* router_w, const float* router_bias, int E, int top_k,
+                       int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                       size_t ws_bytes, void* stream) {
+    return forward(false, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, out,
+                   hist, route_out, ws, ws_bytes, stream);
+}
+
+int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L, int layer,
+                        const uint16_t* x, int T, const float* router_w, const float* router_bias, int E, int top_k,
+                        int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                        size_t ws_bytes, void* stream) {
+    return forward(true, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, out,
+                   hist, route_out, ws, ws_bytes, stream);
+}
+
+int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, uint32_t* hist, void* stream) {
+    if (!expert_offsets || !hist) return MOE_ERR_ARG;
+    if (E < 1 || E > MOE_MAX_E || L < 1 || layer < 0 || layer >= L) return MOE_ERR_RANGE;
+    k_hist_add<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(expert_offsets, E, layer, hist);
+    return cuda_rc(cudaGetLastError());
+}
+
+int moe_rank_experts(const uint32_t* hist_host, int L, int E, uint16_t* pairs_out) {
+    if (!hist_host || !pairs_out) return MOE_ERR_ARG;
+    if (L < 1 || E < 1 || E > MOE_MAX_E || L > 65535) return MOE_ERR_RANGE;
+    const int n = L * E;
+    std::vector<int32_t> order(n);
+    for (int i = 0; i < n; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int32_t a, int32_t b) { return hist_host[a] > hist_host[b]; });
+    for (int r = 0; r < n; ++r) {
+        pairs_out[2 * r] = (uint16_t)(order[r] / E);
+        pairs_out[2 * r + 1] = (uint16_t)(order[r] % E);
+    }
+    return MOE_OK;
+}
+
+int moe_last_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_moe_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
+
+const char* moe_strerror(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument: null, misaligned or overlapping pointer";
+        case MOE_ERR_SHAPE: return "unsupported shape: H, I, block, bit width or arena layout";
+        case MOE_ERR_RANGE: return "value out of range: T, E, top_k, L or layer";
+        case MOE_ERR_WS: return "workspace smaller than moe_workspace_bytes()";
+        case MOE_ERR_CUDA: return "CUDA launch or query failed";
+        case MOE_ERR_SLOT: return "a selected expert has no valid arena slot (it contributed zero)";
+        case MOE_ERR_TIMEOUT: return "a bounded device-side wait expired";
+        default: return "unknown error code";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+"""Decode path (T <= 8) through the C ABI against the CPU oracle."""
+import numpy as np
+import pytest
+
+import moe_synth as S
+import oracle as O
+from helpers import Workload, assert_out_close, check_routing, run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def decode_wl(cuda_ok):
+    return Workload(S.config("decode"))
+
+
+def _compare(wl, layer, x, prefill=False, tokens=None):
+    out, res = run_layer(wl, layer, x, prefill=prefill)
+    ref = wl.oracle_layer(layer, x)
+    check_routing(res, ref["idx"], ref["w"], wl.cfg.E)
+    rel = assert_out_close(out, ref["out_f64"])
+    return out, res, ref, rel
+
+
+def test_tiny_decode(cuda_ok):
+    wl = Workload(S.config("tiny"))
+    _compare(wl, 0, wl.x_host())
+
+
+@pytest.mark.parametrize("T", [1, 5])
+def test_decode_full_layer(decode_wl, T):
+    wl = decode_wl
+    x = S.gen_x(wl.cfg, T)
+    _compare(wl, 0, x)
+
+
+@pytest.mark.parametrize("T", [2, 8])
+def test_decode_other_window_sizes(decode_wl, T):
+    wl = decode_wl
+    _compare(wl, 0, S.gen_x(wl.cfg, T, stream_offset=T))
+
+
+def test_decode_mixed_bits_and_bias(cuda_ok):
+    cfg = S.config("tiny", E=32, top_k=10, H=256, I=96, T=6, bits=(2, 4, 2), zipf_s=1.1, router_std=None)
+    wl = Workload(cfg)
+    _compare(wl, 0, wl.x_host())
+
+
+def test_decode_exact_ties_pick_lower_index(cuda_ok):
+    """Duplicate router rows give exactly equal logits: the lower index wins
+    and its slot comes first; a zero token ties every expert."""
+    import torch
+    cfg = S.config("tiny", E=16, top_k=4, H=128, I=64, T=3)
+    wl = Workload(cfg)
+    W = wl.W_host[0].copy()
+    W[9] = W[2]
+    W[12] = W[2]
+    W[5] = W[7]
+    wl.W_host[0] = W
+    wl.W[0] = torch.from_numpy(W).cuda()
+    x = wl.x_host()
+    x[2] = 0  # all logits 0: the k lowest indices, equal weights
+    out, res, ref, _ = _compare(wl, 0, x)
+    assert res["topk_idx"][2].tolist() == [0, 1, 2, 3]
+    assert np.allclose(res["topk_w"][2], 0.25)
+    assert res["n_rechecked"][0] >= 1
+
+
+def test_decode_histogram_accumulates(decode_wl):
+    import torch
+    wl = decode_wl
+    cfg = wl.cfg
+    hist = torch.zeros((1, cfg.E), dtype=torch.int32, device="cuda")
+    ref = np.zeros((1, cfg.E), np.uint32)
+    for i in range(3):
+        x = S.gen_x(cfg, 5, stream_offset=10 + i)
+        out, res = run_layer(wl, 0, x, prefill=False, hist=hist)
+        counts, *_ = O.permutation(res["topk_idx"], cfg.E)
+        O.hist_add(counts, 0, ref)
+    got = hist.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref)
+    assert got.sum() == 3 * 5 * cfg.top_k
+
+
+def test_decode_missing_slot_contributes_zero(cuda_ok):
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    cfg = S.config("tiny", E=16, top_k=4, H=128, I=64, T=3)
+    wl = Workload(cfg)
+    x = wl.x_host()
+    ref = wl.oracle_layer(0, x)
+    e_bad = int(ref["idx"][1, 0])
+    table = wl.slot_table_host.copy()
+    table[e_bad] = -1
+    wl.slot_table = torch.from_numpy(table).cuda()
+    xt = torch.from_numpy(x.view(np.int16)).cuda()
+    out = torch.zeros_like(xt)
+    ws = torch.empty(M.moe_workspace_bytes(3, cfg.E, cfg.top_k, cfg.H, cfg.I), dtype=torch.uint8, device="cuda")
+    M.moe_forward_decode(wl.desc, wl.arena, wl.slot_table, 1, 0, xt, wl.W[0], None, cfg.top_k, True, out, ws=ws)
+    assert M.moe_last_device_error() == M.MOE_ERR_SLOT
+    assert M.moe_last_device_error() == 0  # read clears
+    d, mini, t2 = wl.mini_arena(0, np.unique(ref["idx"]))
+    t2[e_bad] = -1
+    r2 = O.moe_layer(d, mini, t2, 1, 0, x, wl.W_host[0], None, cfg.top_k)
+    assert r2["rc"] == O.ORC_ERR_SLOT
+    assert_out_close(out.cpu().numpy().view(np.uint16), r2["out_f64"])
+
+
+def test_decode_stack_teacher_forced(cuda_ok):
+    """48 layers x 256 experts, 2/2/4-bit, Zipf bias: the oracle chains its own
+    bf16 outputs; every layer of the library gets the oracle's input."""
+    import torch
+    cfg = S.config("decode_stack")
+    wl = Workload(cfg)
+    x = wl.x_host()
+    hist = torch.zeros((cfg.L, cfg.E), dtype=torch.int32, device="cuda")
+    ref_hist = np.zeros((cfg.L, cfg.E), np.uint32)
+    distinct = []
+    for layer in range(cfg.L):
+        out, res = run_layer(wl, layer, x, prefill=False, hist=hist)
+        ref = wl.oracle_layer(layer, x)
+        counts = check_routing(res, ref["idx"], ref["w"], cfg.E)
+        O.hist_add(counts, layer, ref_hist)
+        assert_out_close(out, ref["out_f64"])
+        distinct.append(int((counts > 0).sum()))
+        x = ref["out"]
+    assert np.array_equal(hist.cpu().numpy().view(np.uint32), ref_hist)
+    assert max(distinct) <= cfg.T * cfg.top_k

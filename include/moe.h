@@ -169,6 +169,21 @@ int moe_last_device_error(void* stream);
 /* Static message for a return code. */
 const char* moe_strerror(int code);
 
+/*
+ * Measurement hooks (no counterpart on the source pages; used by the
+ * benchmark).  moe_set_stage_events(events, n): when n >= 5, every later
+ * forward call records the caller's CUDA events (cudaEvent_t, created with
+ * timing enabled) on its stream at the stage boundaries: events[0] before the
+ * router, [1] after grouping, [2] after the first expert stage (gate/up),
+ * [3] after the second (down), [4] after the combine.  n = 0 (or events =
+ * NULL) turns it off.  The setting is process-wide and read at call time, so
+ * a call captured into a CUDA graph records into the events set at capture.
+ * moe_launch_count(): kernels this process has launched through the library
+ * (host-side counter; launches replayed from a captured graph are not added).
+ */
+int moe_set_stage_events(void* const* events, int n);
+uint64_t moe_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

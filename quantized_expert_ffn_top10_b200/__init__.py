@@ -41,7 +41,8 @@ MOE_ERR_WS, MOE_ERR_CUDA, MOE_ERR_SLOT, MOE_ERR_TIMEOUT = -4, -5, -6, -7
 MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T = 8, 8192
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",
-           "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror")
+           "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
+           "moe_set_stage_events", "moe_launch_count")
 
 
 class RouteOut(ctypes.Structure):
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.moe_last_device_error.argtypes = [P]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_strerror.argtypes = [i32]
+        L.moe_set_stage_events.restype = i32
+        L.moe_set_stage_events.argtypes = [P, i32]
+        L.moe_launch_count.restype = ctypes.c_uint64
+        L.moe_launch_count.argtypes = []
         _lib = L
     return _lib
 
@@ -175,3 +180,18 @@ def moe_rank_experts(hist_host):
 
 def moe_last_device_error(stream=None) -> int:
     return int(lib().moe_last_device_error(_stream(stream)))
+
+
+def moe_set_stage_events(events) -> int:
+    """events: list of 5 torch.cuda.Event(enable_timing=True) (or [] to turn off);
+    later forward calls record them at the stage boundaries."""
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()  # make sure the event exists before its handle is taken
+    n = len(events)
+    arr = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in events])
+    return _check(lib().moe_set_stage_events(arr if n else None, n), "moe_set_stage_events", True)
+
+
+def moe_launch_count() -> int:
+    return int(lib().moe_launch_count())

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -51,6 +52,20 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.total = o;
     return w;
 }
+
+// ---------------------------------------------------------------- process state
+
+std::mutex g_mu;
+std::vector<cudaEvent_t> g_stage_ev;  // measurement hook, see moe_set_stage_events
+std::atomic<uint64_t> g_launches{0};
+uint64_t g_init_mask[4] = {0, 0, 0, 0};  // devices whose kernel attributes are set
+
+inline void stage(int i, cudaStream_t st) {
+    std::lock_guard<std::mutex> g(g_mu);
+    if ((int)g_stage_ev.size() > i) cudaEventRecord(g_stage_ev[i], st);
+}
+
+inline void count(int n) { g_launches += (uint64_t)n; }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -127,6 +142,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
     k_perm_count<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
     k_perm_scan<<<1, MOE_MAX_E, 0, st>>>(pa);
     k_perm_scatter<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
+    count(T <= MOE_DECODE_MAX_T ? 5 : 6);
     return cuda_rc(cudaGetLastError());
 }
 
@@ -172,6 +188,29 @@ bool tmap_codes(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_b
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ---------------------------------------------------------------- process state
+
+// Raise the dynamic shared-memory limit of every large-smem kernel, once per
+// device, so that later calls (and graph captures) only launch.
+int ensure_init() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_mu);
+    if (g_init_mask[dev >> 6] >> (dev & 63) & 1ull) return MOE_OK;
+    const int dsm = MOE_DECODE_MAX_T * 8192 * 2, dnm = MOE_DECODE_MAX_T * 4096 * 4;
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t r) { if (r != cudaSuccess) e = r; };
+    chk(set_smem(k_dec_gateup<4, 4>, dsm)); chk(set_smem(k_dec_gateup<2, 2>, dsm));
+    chk(set_smem(k_dec_gateup<2, 4>, dsm)); chk(set_smem(k_dec_gateup<4, 2>, dsm));
+    chk(set_smem(k_dec_down<4>, dnm)); chk(set_smem(k_dec_down<2>, dnm));
+    chk(set_smem(k_prefill_gemm<0, 4, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 2, 2>, PfCfg<0>::SMEM));
+    chk(set_smem(k_prefill_gemm<0, 2, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 4, 2>, PfCfg<0>::SMEM));
+    chk(set_smem(k_prefill_gemm<1, 4, 4>, PfCfg<1>::SMEM)); chk(set_smem(k_prefill_gemm<1, 2, 2>, PfCfg<1>::SMEM));
+    if (e != cudaSuccess || !encoder()) return MOE_ERR_CUDA;
+    g_init_mask[dev >> 6] |= 1ull << (dev & 63);
+    return MOE_OK;
 }
 
 }  // namespace
@@ -231,14 +270,12 @@ int route_for_layer(const LayerCall& c, const Ws& L, bool tiles, Routed& r) {
 template <int BG, int BU>
 void launch_gateup(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
     const int smem = T * a.H * 2;
-    set_smem(k_dec_gateup<BG, BU>, smem);
     k_dec_gateup<BG, BU><<<dim3((a.I + 31) / 32, umax), 32 * DEC_GU_WARPS, smem, st>>>(a);
 }
 
 template <int BD>
 void launch_down(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
     const int smem = T * a.I * 4;
-    set_smem(k_dec_down<BD>, smem);
     k_dec_down<BD><<<dim3((a.H + 31) / 32, umax), 32 * DEC_DN_WARPS, smem, st>>>(a);
 }
 
@@ -246,8 +283,10 @@ int run_decode(const LayerCall& c) {
     const moe_arena_desc* d = c.d;
     const Ws L = ws_layout(c.T, c.E, c.k, d->H, d->I);
     Routed r;
+    stage(0, c.st);
     int rc = route_for_layer(c, L, false, r);
     if (rc) return rc;
+    stage(1, c.st);
     DecodeArgs a{};
     a.arena = c.arena; a.slot_table = c.slot_table; a.slot_bytes = d->slot_bytes; a.n_slots = d->n_slots;
     for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
@@ -263,17 +302,20 @@ int run_decode(const LayerCall& c) {
     else if (d->bits_gate == 2 && d->bits_up == 2) launch_gateup<2, 2>(a, umax, c.T, c.st);
     else if (d->bits_gate == 2) launch_gateup<2, 4>(a, umax, c.T, c.st);
     else launch_gateup<4, 2>(a, umax, c.T, c.st);
+    stage(2, c.st);
     if (d->bits_down == 4) launch_down<4>(a, umax, c.T, c.st);
     else launch_down<2>(a, umax, c.T, c.st);
+    stage(3, c.st);
     k_combine<float><<<dim3((d->H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
         c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, d->H, c.k, c.residual, c.out);
+    stage(4, c.st);
+    count(3);
     return cuda_rc(cudaGetLastError());
 }
 
 template <int MODE, int B0, int B1>
 void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, const PrefillArgs& a,
                  int mtiles, int ntile_max, cudaStream_t st) {
-    set_smem(k_prefill_gemm<MODE, B0, B1>, PfCfg<MODE>::SMEM);
     k_prefill_gemm<MODE, B0, B1><<<dim3(mtiles, ntile_max), PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
 }
 
@@ -283,8 +325,10 @@ int run_prefill(const LayerCall& c) {
     const Ws L = ws_layout(c.T, c.E, c.k, H, I);
     if (!encoder()) return MOE_ERR_CUDA;
     Routed r;
+    stage(0, c.st);
     int rc = route_for_layer(c, L, true, r);
     if (rc) return rc;
+    stage(1, c.st);
     uint16_t* xp = reinterpret_cast<uint16_t*>(c.ws + L.xp);
     uint16_t* h = reinterpret_cast<uint16_t*>(c.ws + L.h);
     uint16_t* y = reinterpret_cast<uint16_t*>(c.ws + L.y);
@@ -309,11 +353,15 @@ int run_prefill(const LayerCall& c) {
     else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
     else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, tg, tu, a, I / PF_BM, nt, c.st);
     else launch_gemm<0, 4, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    stage(2, c.st);
     a.out = y;
     if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
     else launch_gemm<1, 2, 2>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
+    stage(3, c.st);
     k_combine<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
         c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);
+    stage(4, c.st);
+    count(4);
     return cuda_rc(cudaGetLastError());
 }
 
@@ -351,6 +399,8 @@ static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, 
     int rc = check_layer(c, prefill);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
+    rc = ensure_init();
+    if (rc) return rc;
     return prefill ? run_prefill(c) : run_decode(c);
 }
 
@@ -374,6 +424,7 @@ int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, 
     if (!expert_offsets || !hist) return MOE_ERR_ARG;
     if (E < 1 || E > MOE_MAX_E || L < 1 || layer < 0 || layer >= L) return MOE_ERR_RANGE;
     k_hist_add<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(expert_offsets, E, layer, hist);
+    count(1);
     return cuda_rc(cudaGetLastError());
 }
 
@@ -399,6 +450,16 @@ int moe_last_device_error(void* stream) {
     if (cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
     return v;
 }
+
+int moe_set_stage_events(void* const* events, int n) {
+    if (n < 0 || (n > 0 && !events)) return MOE_ERR_ARG;
+    std::lock_guard<std::mutex> g(g_mu);
+    g_stage_ev.clear();
+    for (int i = 0; i < n; ++i) g_stage_ev.push_back(static_cast<cudaEvent_t>(events[i]));
+    return MOE_OK;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 const char* moe_strerror(int code) {
     switch (code) {

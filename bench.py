@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-decode", action="store_true", help="profiling runs: prefill only")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="profiling runs: skip the oracle timing")
     p.add_argument("--prefill-steps", type=int, default=None)
     return p.parse_args()
 
@@ -182,7 +184,11 @@ def time_graphs(layers: Layers, steps: int, warmup: int, dev: int, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     # stage durations of each graph's last replay (all inside the timed region when steps >= NL)
-    stages = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]
+    try:
+        stages = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]
+    except Exception as ex:  # keep the headline even if the stage hook fails
+        print(f"stage events unavailable: {ex}", file=sys.stderr)
+        stages = [[float("nan")] * 4 for _ in evs]
     distinct = [int((layers.offsets[l][1:] - layers.offsets[l][:-1] > 0).sum().item()) for l in range(NL)]
     del graphs
     return ms, stages, distinct, per_call, clk.summary()
@@ -297,7 +303,31 @@ def run_ours(args):
     hbm, tc_burst, tc_sus, src = peaks()
     K, W = args.steps, max(3, args.warmup)
 
+    line = {"metric": METRIC}
+    if args.no_decode:
+        run_prefill_only = True
+    else:
+        run_prefill_only = False
     # ---- decode (headline)
+    if not run_prefill_only:
+        line = decode_section(args, rank, local, world, dist, hbm, src, K, W)
+    prefill_section(args, line, rank, local, world, dist, tc_burst, tc_sus, src, K, W)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not run_prefill_only:
+        dl = Layers(S.config("decode"), 1, rank)
+        secs, n = oracle_sample(dl, 0, 5)
+        line["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores(), "kind": "oracle",
+                                "sample": "one decode window (T=5) of one layer: router over 512 experts, "
+                                          "the selected experts' FFNs, combine"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def decode_section(args, rank, local, world, dist, hbm, src, K, W):
+    import torch
+    import moe_synth as S
     dl = Layers(S.config("decode"), DECODE_LAYERS, rank)
     c = dl.cfg
     ms, stages, distinct, per_call, clk = time_graphs(dl, K, W, local, dist)
@@ -331,8 +361,12 @@ def run_ours(args):
     }
     del dl
     torch.cuda.empty_cache()
+    return line
 
-    # ---- prefill chunk
+
+def prefill_section(args, line, rank, local, world, dist, tc_burst, tc_sus, src, K, W):
+    import torch
+    import moe_synth as S
     if not args.no_prefill:
         pl = Layers(S.config("prefill"), PREFILL_LAYERS, rank)
         cp = pl.cfg
@@ -362,24 +396,14 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2p, "d2h_bytes_per_step": d2p},
             "gpu_launches": pcp * Kp, "clocks": clkp,
         }
-        line["gpu_launches"] += pcp * Kp
-        if rank == 0 and world == 1:
+        line["gpu_launches"] = line.get("gpu_launches", 0) + pcp * Kp
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
             secs, n = oracle_sample(pl, 0, 16)
             line["prefill"]["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores(),
                                                "kind": "oracle",
                                                "sample": "16 tokens of the 8,192-token chunk, full layer"}
         del pl
-    if rank == 0 and world == 1:
-        dl = Layers(S.config("decode"), 1, rank)
-        secs, n = oracle_sample(dl, 0, 5)
-        line["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores(), "kind": "oracle",
-                                "sample": "one decode window (T=5) of one layer: router over 512 experts, "
-                                          "the selected experts' FFNs, combine"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+        torch.cuda.empty_cache()
 
 
 def run_reference(args):

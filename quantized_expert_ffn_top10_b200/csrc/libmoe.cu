@@ -35,9 +35,9 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     auto put = [&](size_t bytes) { size_t r = o; o += al(std::max<size_t>(bytes, 1)); return r; };
     w.idx = put(P * 4);
     w.w = put(P * 4);
-    w.logit = put((size_t)T * E * 4);
-    w.absum = put(small ? (size_t)T * E * 4 : 0);
-    w.cmax = put((size_t)(H + 1) * 4);
+    w.logit = put((size_t)T * E * (small ? 8 : 4));  // fp64 logits for decode windows, fp32 for chunks
+    w.absum = put(small ? (size_t)T * E * 8 : 0);
+    w.cmax = put((size_t)E * 4);                    // router row norms
     w.offsets = put((size_t)(E + 1) * 4);
     w.perm = put(P * 4);
     w.inv = put(P * 4);
@@ -62,7 +62,8 @@ uint64_t g_init_mask[4] = {0, 0, 0, 0};  // devices whose kernel attributes are 
 
 inline void stage(int i, cudaStream_t st) {
     std::lock_guard<std::mutex> g(g_mu);
-    if ((int)g_stage_ev.size() > i) cudaEventRecord(g_stage_ev[i], st);
+    // external: inside a stream capture this becomes an event-record node of the graph
+    if ((int)g_stage_ev.size() > i) cudaEventRecordWithFlags(g_stage_ev[i], st, cudaEventRecordExternal);
 }
 
 inline void count(int n) { g_launches += (uint64_t)n; }
@@ -96,10 +97,8 @@ int check_route_args(const uint16_t* x, int T, int H, const float* W, int E, int
     return MOE_OK;
 }
 
-inline float gamma32(int n) {
-    const double nu = (double)n * 5.9604644775390625e-8;  // n * 2^-24
-    return (float)(nu / (1.0 - nu));
-}
+// gamma_n = n u / (1 - n u): bound factor of a sum whose terms pass through at most n roundings
+inline double gamma_n(int n, double u) { return (double)n * u / (1.0 - (double)n * u); }
 
 inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -109,27 +108,28 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
                  float* w, int32_t* offsets, int32_t* perm, int32_t* nrechk, uint8_t* ws, const Ws& L, bool want_tiles,
                  uint32_t* hist, int layer, cudaStream_t st) {
     const int P = T * k;
-    float* logit = reinterpret_cast<float*>(ws + L.logit);
     int32_t* nr = nrechk ? nrechk : reinterpret_cast<int32_t*>(ws + L.nrechk);
     if (cudaMemsetAsync(nr, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     TopkArgs ta{};
-    ta.x = x; ta.W = W; ta.b = b; ta.logit = logit; ta.idx = idx; ta.w = w; ta.n_rechecked = nr;
+    ta.x = x; ta.W = W; ta.b = b; ta.logit = ws + L.logit; ta.idx = idx; ta.w = w; ta.n_rechecked = nr;
     ta.T = T; ta.H = H; ta.E = E; ta.k = k;
+    const int tk_grid = (T + MOE_TOPK_WARPS - 1) / MOE_TOPK_WARPS;
     if (T <= MOE_DECODE_MAX_T) {
-        float* absum = reinterpret_cast<float*>(ws + L.absum);
+        double* logit = reinterpret_cast<double*>(ws + L.logit);
+        double* absum = reinterpret_cast<double*>(ws + L.absum);
         k_router_gemv<<<(E + 7) / 8, 256, 0, st>>>(x, T, H, W, b, E, logit, absum);
         ta.absum = absum;
-        ta.gamma32 = gamma32(H / 32 + 6);
+        ta.gfast = gamma_n(H / 32 + 6, 1.1102230246251565e-16);
+        k_topk<true><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     } else {
-        unsigned int* cmax = reinterpret_cast<unsigned int*>(ws + L.cmax);
-        if (cudaMemsetAsync(cmax, 0, (size_t)(H + 1) * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
-        k_router_colmax<<<dim3((H + 1 + 255) / 256, (E + 31) / 32), 256, 0, st>>>(W, b, E, H, cmax);
+        float* wnorm = reinterpret_cast<float*>(ws + L.cmax);
+        float* logit = reinterpret_cast<float*>(ws + L.logit);
+        k_router_norms<<<(E + 7) / 8, 256, 0, st>>>(W, E, H, wnorm);
         k_router_gemm<<<dim3((E + RG_BN - 1) / RG_BN, (T + RG_BM - 1) / RG_BM), 256, 0, st>>>(x, T, H, W, b, E, logit);
-        ta.absum = nullptr;
-        ta.cmax = cmax;
-        ta.gamma32 = gamma32(H + 2);
+        ta.wnorm = wnorm;
+        ta.gfast = gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);
+        k_topk<false><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     }
-    k_topk<<<(T + MOE_TOPK_WARPS - 1) / MOE_TOPK_WARPS, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     PermArgs pa{};
     pa.idx = idx; pa.P = P; pa.E = E; pa.nchunks = (P + PERM_CHUNK - 1) / PERM_CHUNK;
     pa.chunk_cnt = reinterpret_cast<int32_t*>(ws + L.chunk);
@@ -316,7 +316,8 @@ int run_decode(const LayerCall& c) {
 template <int MODE, int B0, int B1>
 void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, const PrefillArgs& a,
                  int mtiles, int ntile_max, cudaStream_t st) {
-    k_prefill_gemm<MODE, B0, B1><<<dim3(mtiles, ntile_max), PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
+    (void)mtiles;  // each CTA walks all M-tiles of its N-tile
+    k_prefill_gemm<MODE, B0, B1><<<ntile_max, PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
 }
 
 int run_prefill(const LayerCall& c) {

@@ -11,33 +11,38 @@
 //   GEMM2: D = W_d[rows] h^T                           (K = I)
 //          Y[pair][row] = bf16(w_pair * D)
 //
-// Roles (384 threads): warp 0 issues TMA loads of the activation tile (128-B
-// swizzled) and of the raw code tile of each weight matrix; warp 1 owns TMEM
-// and one of its threads issues tcgen05.mma; warps 4-11 dequantise codes to
-// bf16 straight into the 128-B swizzled K-major layout the MMA reads, then run
-// the epilogue from TMEM.  Stages cycle through full / dequantised / empty
-// mbarriers; every wait is bounded.
+// A CTA owns one N-tile and walks all M-tiles, so the activation rows stay in
+// L2 and setup is paid once.  Roles (448 threads): warp 0 issues TMA loads of
+// the activation tile (128-B swizzled) and of the raw code tile of each weight
+// matrix (one 3-D tensor map spans all arena slots); warp 1 owns TMEM and one
+// of its threads issues tcgen05.mma; warps 2-5 drain finished accumulators
+// (TMEM -> registers -> global; the down GEMM double-buffers them so this
+// overlaps the next M-tile); warps 6-13 dequantise codes to bf16 straight into
+// the 128-B swizzled K-major layout the MMA reads.  Stages cycle through full /
+// dequantised / empty mbarriers; every wait is bounded.
 #pragma once
 #include "common.cuh"
 
 #define PF_BK 64          // K elements per stage (one 128-byte swizzle row of bf16)
-#define PF_BM 128         // weight rows per tile
+#define PF_BM 128         // weight rows per M-tile
 #define PF_BN_MAX 256     // pair rows per tile
 #define PF_BOX_ROWS 16    // activation rows per TMA box
-#define PF_THREADS 384
-#define PF_DQ_WARP0 4     // first dequant / epilogue warp
+#define PF_EPI_WARP0 2    // epilogue warps 2..5 (TMEM lane quadrants 2, 3, 0, 1)
+#define PF_DQ_WARP0 6     // dequantisation warps 6..13
 #define PF_DQ_THREADS 256
+#define PF_THREADS 448
 
 template <int MODE>  // 0 = gate/up + SwiGLU, 1 = down + gate weight
 struct PfCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
     static constexpr int STAGES = MODE == 0 ? 3 : 4;
+    static constexpr int NACC = MODE == 0 ? 1 : 2;               // accumulator buffers in TMEM
     static constexpr int A_BYTES = PF_BM * PF_BK * 2;            // one dequantised matrix tile
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int C_BYTES = PF_BM * PF_BK / 2;            // raw codes (<= 4-bit)
     static constexpr int STAGE_BYTES = NMAT * A_BYTES + B_BYTES + NMAT * C_BYTES;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-    static constexpr int TMEM_COLS = MODE == 0 ? 512 : 256;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*gate weights*/ + 256 /*barriers*/;
+    static constexpr int TMEM_COLS = 512;
 };
 
 struct PrefillArgs {
@@ -54,63 +59,87 @@ struct PrefillArgs {
     uint16_t* out;           // GEMM1: h [P][I]; GEMM2: Y [P][H]
 };
 
-// codes of 8 consecutive 4-bit (or 2-bit) elements -> 8 dequantised bf16 (uint4)
+// 8 codes (one 32-bit word of 4-bit codes, or 16 bits of 2-bit codes) ->
+// 8 bf16 weights s * (q - offset), each rounded once from the exact product.
+// q - offset is formed exactly in bf16 (128 + q by an exponent-bias bit
+// pattern, then a subtraction).  The fp16 scale splits exactly into bf16
+// s_hi + s_lo (11 significant bits = 8 + 3), (q - offset) * s_lo is exact,
+// and one fused multiply-add adds (q - offset) * s_hi with a single rounding.
 template <int BITS>
-__device__ __forceinline__ uint4 dq8(uint32_t w, float s) {
-    constexpr float kMagic = 8388608.0f + (float)(1 << (BITS - 1));  // 2^23 + offset
-    float f[8];
+__device__ __forceinline__ uint4 dq8(uint32_t w, uint32_t s2hi, uint32_t s2lo) {
+    constexpr uint32_t kMagic = 0x43004300u;                       // bf16 pair (128, 128)
+    constexpr uint32_t kOff = BITS == 4 ? 0x43084308u : 0x43024302u;  // bf16 pair (136, 136) or (130, 130)
+    uint32_t pr[4];
+    // byte_perm selector: result byte 0 <- byte i of the first word, byte 2 <- byte i of the second
+    if (BITS == 4) {
+        // pair i = (low nibble, high nibble) of byte i
+        const uint32_t w4 = w >> 4;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t q = (w >> (BITS * i)) & ((1u << BITS) - 1);
-        f[i] = (__uint_as_float(0x4B000000u | q) - kMagic) * s;  // exact (q - offset) * s, one rounding
+        for (int i = 0; i < 4; ++i) pr[i] = (__byte_perm(w, w4, (uint32_t)(i | ((4 + i) << 8))) & 0x000F000Fu) | kMagic;
+    } else {
+        // byte i holds 4 codes at bit pairs 0-1, 2-3, 4-5, 6-7
+        const uint32_t w2 = w >> 2, w4 = w >> 4, w6 = w >> 6;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            pr[2 * i] = (__byte_perm(w, w2, (uint32_t)(i | ((4 + i) << 8))) & 0x00030003u) | kMagic;
+            pr[2 * i + 1] = (__byte_perm(w4, w6, (uint32_t)(i | ((4 + i) << 8))) & 0x00030003u) | kMagic;
+        }
     }
     uint4 r;
-    r.x = pack_bf16x2(f[0], f[1]);
-    r.y = pack_bf16x2(f[2], f[3]);
-    r.z = pack_bf16x2(f[4], f[5]);
-    r.w = pack_bf16x2(f[6], f[7]);
+    uint32_t* rr = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&pr[i]);
+        __nv_bfloat162 o = *reinterpret_cast<const __nv_bfloat162*>(&kOff);
+        __nv_bfloat162 shi = *reinterpret_cast<__nv_bfloat162*>(&s2hi);
+        __nv_bfloat162 slo = *reinterpret_cast<__nv_bfloat162*>(&s2lo);
+        __nv_bfloat162 q = __hsub2(v, o);                    // exact: small integers
+        __nv_bfloat162 d = __hfma2(q, shi, __hmul2(q, slo));  // exact low part, one rounding
+        rr[i] = *reinterpret_cast<uint32_t*>(&d);
+    }
     return r;
 }
 
 // One 32-element block of one row: codes from the staging tile -> 4 swizzled
-// 16-byte chunks of the A tile.
+// 16-byte chunks of the A tile (row r at r * 128 B, chunk j at (j ^ (r & 7)) * 16).
 template <int BITS>
 __device__ __forceinline__ void dequant_unit(const uint8_t* ctile, uint8_t* atile, int row, int half, float s) {
     constexpr int ROWB = PF_BK * BITS / 8;  // staged code bytes per row
     const uint8_t* src = ctile + row * ROWB + half * (32 * BITS / 8);
-    uint32_t w[BITS];  // 32 codes = BITS words
+    uint32_t w[4];
     if (BITS == 4) {
         uint4 v = *reinterpret_cast<const uint4*>(src);
         w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     } else {
         uint2 v = *reinterpret_cast<const uint2*>(src);
-        w[0] = v.x; w[1] = v.y;
+        w[0] = v.x & 0xffffu; w[1] = v.x >> 16; w[2] = v.y & 0xffffu; w[3] = v.y >> 16;
     }
+    const float shi = __bfloat162float(__float2bfloat16_rn(s));
+    const uint32_t s2hi = pack_bf16x2(shi, shi), s2lo = pack_bf16x2(s - shi, s - shi);  // both exact
     uint8_t* rowp = atile + row * 128;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        // chunk cc holds elements 8cc..8cc+7 of this block
-        uint32_t codes = (BITS == 4) ? w[cc] : ((w[cc >> 1] >> (16 * (cc & 1))) & 0xffffu);
-        uint4 v = dq8<BITS>(codes, s);
-        int j = half * 4 + cc;
-        *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = v;
+    for (int cc = 0; cc < 4; ++cc) {  // chunk cc holds elements 8cc..8cc+7 of this block
+        const int j = half * 4 + cc;
+        *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = dq8<BITS>(w[cc], s2hi, s2lo);
     }
 }
 
+// One CTA per N-tile (expert e, rows row0 .. row0+nrows of the grouped
+// activations); it walks every M-tile of the output features.  Stage i covers
+// (M-tile i / nk, K-block i % nk).
 template <int MODE, int B0, int B1>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     k_prefill_gemm(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC0,
                    const __grid_constant__ CUtensorMap tmC1, PrefillArgs a) {
     using C = PfCfg<MODE>;
-    const int tile = blockIdx.y;
+    const int tile = blockIdx.x;
     if (tile >= a.meta[1]) return;
     const int4 td = a.tiles[tile];
     const int e = td.x, row0 = td.y, nrows = td.z;
     const int npad = (nrows + 15) & ~15;
-    const int mt = blockIdx.x;
     const int K = MODE == 0 ? a.H : a.I;
     const int NOUT = MODE == 0 ? a.I : a.H;  // output features (row length of `out`)
-    const int nk = K / PF_BK;
+    const int nk = K / PF_BK, nmt = NOUT / PF_BM, nstage = nk * nmt;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     extern __shared__ uint8_t smem_raw[];
@@ -118,20 +147,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint8_t* sB = smem;                                          // [STAGES][B_BYTES]
     uint8_t* sA = sB + C::STAGES * C::B_BYTES;                   // [STAGES][NMAT][A_BYTES]
     uint8_t* sC = sA + C::STAGES * C::NMAT * C::A_BYTES;         // [STAGES][NMAT][C_BYTES]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::STAGES * C::NMAT * C::C_BYTES);
+    float* s_w = reinterpret_cast<float*>(sC + C::STAGES * C::NMAT * C::C_BYTES);  // [256] gate weights
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + PF_BN_MAX);
     uint64_t* full = bars;                   // TMA bytes landed
     uint64_t* deq = bars + C::STAGES;        // dequantised A written
     uint64_t* empty = bars + 2 * C::STAGES;  // MMA finished reading the stage
-    uint64_t* accf = bars + 3 * C::STAGES;   // accumulators final
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+    uint64_t* accf = bars + 3 * C::STAGES;   // [NACC] accumulator final
+    uint64_t* acce = accf + C::NACC;         // [NACC] accumulator drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + C::NACC);
 
     const int64_t slot = a.slot_table[(int64_t)a.layer * a.E + e];
     if (slot < 0 || slot >= a.n_slots) {  // expert without weights contributes zero
-        if (threadIdx.x == 0 && mt == 0) moe_set_status(MOE_ERR_SLOT);
-        for (int i = threadIdx.x; i < nrows * PF_BM; i += blockDim.x) {
-            int n = i / PF_BM, r = i % PF_BM;
-            a.out[(size_t)(row0 + n) * NOUT + mt * PF_BM + r] = 0;
-        }
+        if (threadIdx.x == 0) moe_set_status(MOE_ERR_SLOT);
+        for (int i = threadIdx.x; i < nrows * NOUT; i += blockDim.x)
+            a.out[(size_t)(row0 + i / NOUT) * NOUT + i % NOUT] = 0;
         return;
     }
 
@@ -141,9 +170,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             mbar_init(&deq[s], PF_DQ_THREADS / 32);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < C::NACC; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+        }
         fence_mbar_init();
     }
+    if (MODE == 1)
+        for (int n = threadIdx.x; n < nrows; n += blockDim.x) s_w[n] = __ldg(a.topk_w + a.perm[row0 + n]);
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -160,96 +194,103 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             tma_prefetch_desc(&tmC0);
             if (C::NMAT == 2) tma_prefetch_desc(&tmC1);
             const uint32_t bytes = npad * PF_BK * 2 + PF_BM * PF_BK * B0 / 8 + (C::NMAT == 2 ? PF_BM * PF_BK * B1 / 8 : 0);
-            for (int i = 0; i < nk && alive; ++i) {
+            for (int i = 0; i < nstage && alive; ++i) {
                 const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
+                const int kb = i % nk, rowbase = (i / nk) * PF_BM;
                 if (!mbar_wait(&empty[s], ph ^ 1)) { alive = false; break; }
                 mbar_arrive_expect_tx(&full[s], bytes);
                 for (int r = 0; r < npad; r += PF_BOX_ROWS)
-                    tma_load_2d(sB + s * C::B_BYTES + r * 128, &tmB, &full[s], i * PF_BK, row0 + r);
-                const int rowbase = mt * PF_BM;
+                    tma_load_2d(sB + s * C::B_BYTES + r * 128, &tmB, &full[s], kb * PF_BK, row0 + r);
                 asm volatile(
                     "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
                         "r"(smem_u32(sC + (s * C::NMAT + 0) * C::C_BYTES)), "l"(&tmC0), "r"(smem_u32(&full[s])),
-                    "r"(i * PF_BK * B0 / 8), "r"(rowbase), "r"((int)slot)
+                    "r"(kb * PF_BK * B0 / 8), "r"(rowbase), "r"((int)slot)
                     : "memory");
                 if (C::NMAT == 2)
                     asm volatile(
                         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
                             "r"(smem_u32(sC + (s * C::NMAT + 1) * C::C_BYTES)), "l"(&tmC1), "r"(smem_u32(&full[s])),
-                        "r"(i * PF_BK * B1 / 8), "r"(rowbase), "r"((int)slot)
+                        "r"(kb * PF_BK * B1 / 8), "r"(rowbase), "r"((int)slot)
                         : "memory");
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = make_idesc_bf16(PF_BM, npad);
-            for (int i = 0; i < nk && alive; ++i) {
-                const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
-                if (!mbar_wait(&full[s], ph) || !mbar_wait(&deq[s], ph)) { alive = false; break; }
+            for (int mt = 0; mt < nmt && alive; ++mt) {
+                const int buf = mt % C::NACC, use = mt / C::NACC;
+                if (!mbar_wait(&acce[buf], (use & 1) ^ 1)) { alive = false; break; }  // drained by the epilogue
                 tc_fence_after();
-                const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
+                const uint32_t dcol = tmem + buf * 256;
+                for (int kb = 0; kb < nk; ++kb) {
+                    const int i = mt * nk + kb;
+                    const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
+                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&deq[s], ph)) { alive = false; break; }
+                    tc_fence_after();
+                    const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < PF_BK / 16; ++kk) {
-                    const uint64_t bdesc = make_sdesc_sw128(bb + kk * 32);
+                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
+                        const uint64_t bdesc = make_sdesc_sw128(bb + kk * 32);
 #pragma unroll
-                    for (int m = 0; m < C::NMAT; ++m) {
-                        const uint32_t ab = smem_u32(sA + (s * C::NMAT + m) * C::A_BYTES);
-                        tc_mma_bf16(tmem + m * 256, make_sdesc_sw128(ab + kk * 32), bdesc, idesc, (i | kk) != 0);
+                        for (int m = 0; m < C::NMAT; ++m) {
+                            const uint32_t ab = smem_u32(sA + (s * C::NMAT + m) * C::A_BYTES);
+                            tc_mma_bf16(dcol + m * 256, make_sdesc_sw128(ab + kk * 32), bdesc, idesc, (kb | kk) != 0);
+                        }
                     }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                tc_commit(&accf[buf]);
             }
-            tc_commit(accf);
         }
     } else if (warp >= PF_DQ_WARP0) {
         const int dt = threadIdx.x - PF_DQ_WARP0 * 32;  // 0..255
         const int row = dt >> 1, half = dt & 1;
-        const int grow = mt * PF_BM + row;  // weight row in the matrix
-        const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(a.arena + slot * a.slot_bytes +
-                                                               a.off_scales[MODE == 0 ? 0 : 2]) +
-                              (size_t)grow * (K / 32);
-        const uint16_t* sc1 =
-            reinterpret_cast<const uint16_t*>(a.arena + slot * a.slot_bytes + a.off_scales[1]) + (size_t)grow * (K / 32);
-        for (int i = 0; i < nk; ++i) {
+        const uint8_t* sbase = a.arena + slot * a.slot_bytes;
+        const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[MODE == 0 ? 0 : 2]);
+        const uint16_t* sc1 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[1]);
+        for (int i = 0; i < nstage; ++i) {
             const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
+            const int kb = i % nk;
+            const size_t grow = (size_t)((i / nk) * PF_BM + row);  // weight row in the matrix
+            const uint16_t q0 = __ldg(sc0 + grow * (K / 32) + 2 * kb + half);
+            const uint16_t q1 = C::NMAT == 2 ? __ldg(sc1 + grow * (K / 32) + 2 * kb + half) : 0;
             if (!mbar_wait(&full[s], ph)) { alive = false; break; }
-            const float s0 = half_bits_to_f32(__ldg(sc0 + 2 * i + half));
-            dequant_unit<B0>(sC + (s * C::NMAT + 0) * C::C_BYTES, sA + (s * C::NMAT + 0) * C::A_BYTES, row, half, s0);
-            if (C::NMAT == 2) {
-                const float s1 = half_bits_to_f32(__ldg(sc1 + 2 * i + half));
+            dequant_unit<B0>(sC + (s * C::NMAT + 0) * C::C_BYTES, sA + (s * C::NMAT + 0) * C::A_BYTES, row, half,
+                             half_bits_to_f32(q0));
+            if (C::NMAT == 2)
                 dequant_unit<B1>(sC + (s * C::NMAT + 1) * C::C_BYTES, sA + (s * C::NMAT + 1) * C::A_BYTES, row, half,
-                                 s1);
-            }
+                                 half_bits_to_f32(q1));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&deq[s]);
         }
-        // epilogue: TMEM -> registers -> global
-        if (alive && mbar_wait(accf, 0)) {
+    } else {  // epilogue warps: TMEM -> registers -> global, one M-tile at a time
+        const int q = warp & 3;  // TMEM lane quadrant this warp may read
+        for (int mt = 0; mt < nmt && alive; ++mt) {
+            const int buf = mt % C::NACC, use = mt / C::NACC;
+            if (!mbar_wait(&accf[buf], use & 1)) { alive = false; break; }
             tc_fence_after();
-            const int q = warp & 3;              // TMEM lane quadrant this warp may read
-            const int chalf = (warp - PF_DQ_WARP0) >> 2;
             const int r = mt * PF_BM + q * 32 + lane;  // output feature of this thread
-            for (int c0 = chalf * 16; c0 < npad; c0 += 32) {
+            const uint32_t ta0 = tmem + buf * 256 + ((uint32_t)(q * 32) << 16);
+            for (int c0 = 0; c0 < npad; c0 += 16) {
                 uint32_t v0[16], v1[16];
-                const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + c0;
-                tmem_ld16(ta, v0);
-                if (MODE == 0) tmem_ld16(ta + 256, v1);
+                tmem_ld16(ta0 + c0, v0);
+                if (MODE == 0) tmem_ld16(ta0 + 256 + c0, v1);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int n = c0 + j;
                     if (n < nrows) {
                         float o;
-                        if (MODE == 0) {
-                            o = silu_f32(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
-                        } else {
-                            o = __ldg(a.topk_w + a.perm[row0 + n]) * __uint_as_float(v0[j]);
-                        }
+                        if (MODE == 0) o = silu_f32(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
+                        else o = s_w[n] * __uint_as_float(v0[j]);
                         a.out[(size_t)(row0 + n) * NOUT + r] = f32_to_bf16_bits(o);
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
         }
     }
     tc_fence_before();

@@ -18,56 +18,37 @@
 #define MOE_TOPK_WARPS 4
 #define MOE_CAND_EXTRA 2  // fp64 candidates beyond k
 
-// ---------------------------------------------------------------- column max for the prefill bound
+// ---------------------------------------------------------------- decode router: fp64 GEMV, warp per expert
 
-// cmax[h] = max_e |W[e][h]| (h < H), cmax[H] = max_e |b_e|, as float bits.
-// The caller zeroes cmax first; all values are >= 0 so unsigned max is exact.
-__global__ void k_router_colmax(const float* __restrict__ W, const float* __restrict__ b, int E, int H,
-                                unsigned int* __restrict__ cmax) {
-    int h = blockIdx.x * blockDim.x + threadIdx.x;
-    int e0 = blockIdx.y * 32, e1 = min(E, e0 + 32);
-    if (h < H) {
-        float m = 0.f;
-        for (int e = e0; e < e1; ++e) m = fmaxf(m, fabsf(__ldg(W + (size_t)e * H + h)));
-        atomicMax(cmax + h, __float_as_uint(m));
-    } else if (h == H && b != nullptr) {
-        float m = 0.f;
-        for (int e = e0; e < e1; ++e) m = fmaxf(m, fabsf(b[e]));
-        atomicMax(cmax + H, __float_as_uint(m));
-    }
-}
-
-// ---------------------------------------------------------------- decode router: GEMV, warp per expert
-
-// Fast logits and per-entry bounds for T <= MOE_DECODE_MAX_T tokens.  Lane L
-// sums h = 4L + 128i + j sequentially (chain H/32), then a 5-level butterfly
-// and the bias: chain length H/32 + 6.  absum[t][e] = sum |x W| + |b|.
+// Logits in fp64 for T <= MOE_DECODE_MAX_T tokens, with per-entry bound sums.
+// Lane L sums h = 4L + 128i + j sequentially (chain H/32), then a 5-level
+// butterfly and the bias: chain length H/32 + 6.  absum[t][e] = sum |x W| + |b|.
+// fp64 costs nothing here: the kernel is bound by reading W (4 B per weight).
 __global__ void __launch_bounds__(256) k_router_gemv(const uint16_t* __restrict__ x, int T, int H,
                                                      const float* __restrict__ W, const float* __restrict__ b,
-                                                     int E, float* __restrict__ logit, float* __restrict__ absum) {
+                                                     int E, double* __restrict__ logit, double* __restrict__ absum) {
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (e >= E) return;
-    float acc[MOE_DECODE_MAX_T], ab[MOE_DECODE_MAX_T];
+    double acc[MOE_DECODE_MAX_T], ab[MOE_DECODE_MAX_T];
 #pragma unroll
-    for (int t = 0; t < MOE_DECODE_MAX_T; ++t) acc[t] = ab[t] = 0.f;
+    for (int t = 0; t < MOE_DECODE_MAX_T; ++t) acc[t] = ab[t] = 0.0;
     const float4* w4 = reinterpret_cast<const float4*>(W + (size_t)e * H);
+#pragma unroll 2
     for (int i = lane; i < H / 4; i += 32) {
         float4 w = __ldg(w4 + i);
+        const double w0 = w.x, w1 = w.y, w2 = w.z, w3 = w.w;
 #pragma unroll
         for (int t = 0; t < MOE_DECODE_MAX_T; ++t) {
             if (t < T) {
                 uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)t * H) + i);
-                float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
-                float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
-                acc[t] = fmaf(x0, w.x, acc[t]);
-                acc[t] = fmaf(x1, w.y, acc[t]);
-                acc[t] = fmaf(x2, w.z, acc[t]);
-                acc[t] = fmaf(x3, w.w, acc[t]);
-                ab[t] = fmaf(fabsf(x0), fabsf(w.x), ab[t]);
-                ab[t] = fmaf(fabsf(x1), fabsf(w.y), ab[t]);
-                ab[t] = fmaf(fabsf(x2), fabsf(w.z), ab[t]);
-                ab[t] = fmaf(fabsf(x3), fabsf(w.w), ab[t]);
+                const double x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+                const double x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+                acc[t] = fma(x0, w0, acc[t]);
+                acc[t] = fma(x1, w1, acc[t]);
+                acc[t] = fma(x2, w2, acc[t]);
+                acc[t] = fma(x3, w3, acc[t]);
+                ab[t] += fabs(x0 * w0) + fabs(x1 * w1) + fabs(x2 * w2) + fabs(x3 * w3);
             }
         }
     }
@@ -80,12 +61,30 @@ __global__ void __launch_bounds__(256) k_router_gemv(const uint16_t* __restrict_
         }
     }
     if (lane == 0) {
-        float bb = b ? b[e] : 0.f;
+        double bb = b ? (double)b[e] : 0.0;
         for (int t = 0; t < T; ++t) {
             logit[(size_t)t * E + e] = acc[t] + bb;
-            absum[(size_t)t * E + e] = ab[t] + fabsf(bb);
+            absum[(size_t)t * E + e] = ab[t] + fabs(bb);
         }
     }
+}
+
+// ---------------------------------------------------------------- router weight row norms
+
+// wnorm[e] >= ||W[e]||_2 (fp32, inflated by 0.1% to cover its own rounding)
+__global__ void k_router_norms(const float* __restrict__ W, int E, int H, float* __restrict__ wnorm) {
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (e >= E) return;
+    const float4* w4 = reinterpret_cast<const float4*>(W + (size_t)e * H);
+    float s = 0.f;
+    for (int i = lane; i < H / 4; i += 32) {
+        float4 w = __ldg(w4 + i);
+        s = fmaf(w.x, w.x, fmaf(w.y, w.y, fmaf(w.z, w.z, fmaf(w.w, w.w, s))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) wnorm[e] = sqrtf(s) * 1.001f;
 }
 
 // ---------------------------------------------------------------- prefill router: fp32 tiled GEMM
@@ -94,8 +93,9 @@ __global__ void __launch_bounds__(256) k_router_gemv(const uint16_t* __restrict_
 #define RG_BN 64
 #define RG_BK 16
 
-// l[t][e] = sum_h x[t][h] W[e][h] + b_e, each output summed sequentially over
-// h by one thread (chain length H + 1).
+// l[t][e] = sum_h x[t][h] W[e][h] + b_e.  Each output is summed by one thread
+// in blocks: 16 products into a fresh partial, partials added in order, then
+// the bias, so no product passes through more than 16 + H/16 + 1 roundings.
 __global__ void __launch_bounds__(256) k_router_gemm(const uint16_t* __restrict__ x, int T, int H,
                                                      const float* __restrict__ W, const float* __restrict__ b,
                                                      int E, float* __restrict__ logit) {
@@ -137,6 +137,11 @@ __global__ void __launch_bounds__(256) k_router_gemm(const uint16_t* __restrict_
             xa = xok ? __ldg(reinterpret_cast<const uint4*>(xp + k0 + RG_BK)) : make_uint4(0, 0, 0, 0);
             wa = wok ? __ldg(reinterpret_cast<const float4*>(wp + k0 + RG_BK)) : make_float4(0, 0, 0, 0);
         }
+        float part[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < RG_BK; ++kk) {
             float4 a0 = *reinterpret_cast<const float4*>(&Xs[kk][ty * 8]);
@@ -147,8 +152,12 @@ __global__ void __launch_bounds__(256) k_router_gemm(const uint16_t* __restrict_
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], bb[j], part[i][j]);
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -165,37 +174,18 @@ __global__ void __launch_bounds__(256) k_router_gemm(const uint16_t* __restrict_
 // ---------------------------------------------------------------- certified top-k
 
 struct TopkArgs {
-    const uint16_t* x;       // [T][H] bf16
-    const float* W;          // [E][H]
-    const float* b;          // [E] or null
-    const float* logit;      // [T][E] fast fp32 logits
-    const float* absum;      // [T][E] per-entry bound sums, or null -> use cmax
-    const unsigned int* cmax;  // [H+1] column maxima (float bits), used when absum == null
-    int32_t* idx;            // [T][k]
-    float* w;                // [T][k]
-    int32_t* n_rechecked;    // [1] or null
-    float gamma32;           // bound factor of the fast logits: n u / (1 - n u)
+    const uint16_t* x;      // [T][H] bf16
+    const float* W;         // [E][H]
+    const float* b;         // [E] or null
+    const void* logit;      // [T][E]: double (decode) or float (prefill) fast logits
+    const double* absum;    // decode: [T][E] sums of |x W| + |b|
+    const float* wnorm;     // prefill: [E] upper bounds of ||W[e]||_2
+    int32_t* idx;           // [T][k]
+    float* w;               // [T][k]
+    int32_t* n_rechecked;   // [1]
+    double gfast;           // gamma_n of the fast logits' summation
     int T, H, E, k;
 };
-
-// warp-wide argmax of (v desc, e asc); every lane returns the winner
-__device__ __forceinline__ void warp_best(float& v, int& e) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        float v2 = __shfl_xor_sync(0xffffffffu, v, o);
-        int e2 = __shfl_xor_sync(0xffffffffu, e, o);
-        if (v2 > v || (v2 == v && e2 < e)) { v = v2; e = e2; }
-    }
-}
-
-__device__ __forceinline__ void warp_best_d(double& v, int& e) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        double v2 = __shfl_xor_sync(0xffffffffu, v, o);
-        int e2 = __shfl_xor_sync(0xffffffffu, e, o);
-        if (v2 > v || (v2 == v && e2 < e)) { v = v2; e = e2; }
-    }
-}
 
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
@@ -203,36 +193,68 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     return v;
 }
 
-// fp64 logit of expert e for token t, summed over lane-strided chains of
-// length H/32 and a 5-level butterfly; also returns sum |x W| + |b|.
-__device__ __forceinline__ void logit_fp64_parallel(const TopkArgs& a, int t, int e, double& v, double& ab) {
-    const int lane = threadIdx.x & 31;
-    const uint16_t* xr = a.x + (size_t)t * a.H;
-    const float* wr = a.W + (size_t)e * a.H;
-    double s = 0.0, sa = 0.0;
-    for (int h = lane; h < a.H; h += 32) {
-        double p = (double)bf16_bits_to_f32(xr[h]) * (double)__ldg(wr + h);
-        s += p;
-        sa += fabs(p);
-    }
-    s = warp_sum_d(s);
-    sa = warp_sum_d(sa);
-    double bb = a.b ? (double)a.b[e] : 0.0;
-    v = s + bb;
-    ab = sa + fabs(bb);
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
 }
 
-// The definition: fp64, sequential over h, then + b.  One thread.
+__device__ __forceinline__ double warp_min_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// The definition: fp64, sequential over h, then + b (one thread).
 __device__ __forceinline__ double logit_fp64_exact(const TopkArgs& a, int t, int e) {
     const uint16_t* xr = a.x + (size_t)t * a.H;
     const float* wr = a.W + (size_t)e * a.H;
     double s = 0.0;
+#pragma unroll 8
     for (int h = 0; h < a.H; ++h) s = fma((double)bf16_bits_to_f32(xr[h]), (double)__ldg(wr + h), s);
     if (a.b) s += (double)a.b[e];
     return s;
 }
 
-// One warp per token.  Lanes hold logits of experts e = lane + 32 i.
+// Lanes j < M hold (cval, cbnd, ce).  Sort them by (cval desc, ce asc); lane r
+// receives position r.  Returns whether every decision is certified: each of
+// the first k positions is separated from the next, and position k-1 clears
+// `rest` (the upper end of everything outside the candidates).
+__device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int& ce, int M, int k, double rest) {
+    const int lane = threadIdx.x & 31;
+    int rank = 0;
+    for (int j = 0; j < M; ++j) {
+        double oj = __shfl_sync(0xffffffffu, cval, j);
+        int ej = __shfl_sync(0xffffffffu, ce, j);
+        if (lane < M && (oj > cval || (oj == cval && ej < ce))) ++rank;
+    }
+    int src = 0;
+    for (int j = 0; j < M; ++j)
+        if (__shfl_sync(0xffffffffu, rank, j) == lane) src = j;
+    cval = __shfl_sync(0xffffffffu, cval, src);
+    cbnd = __shfl_sync(0xffffffffu, cbnd, src);
+    ce = __shfl_sync(0xffffffffu, ce, src);
+    const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
+    const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
+    bool ok = true;
+    if (lane < k && lane + 1 < M) ok = (cval - cbnd) > (nv + nb);
+    if (lane == k - 1) ok = ok && (rest == -INFINITY || (cval - cbnd) > rest);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void write_topk(const TopkArgs& a, int t, double cval, int ce) {
+    const int lane = threadIdx.x & 31;
+    const double v0 = __shfl_sync(0xffffffffu, cval, 0);
+    const double z = (lane < a.k) ? exp(cval - v0) : 0.0;
+    const double zs = warp_sum_d(z);
+    if (lane < a.k) {
+        a.idx[(size_t)t * a.k + lane] = ce;
+        a.w[(size_t)t * a.k + lane] = (float)(z / zs);
+    }
+}
+
+// One warp per token; lanes hold the fast logits of experts e = lane + 32 i.
+template <bool F64>
 __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
     __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
     __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
@@ -241,153 +263,155 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
     if (t >= a.T) return;
     const int E = a.E, k = a.k, H = a.H;
     constexpr int NV = MOE_MAX_E / 32;
-    const double u64 = 1.1102230246251565e-16;  // 2^-53
-    // oracle's own rounding bound (sequential fp64, chain H + 1) per unit of B
-    const double g_or = (double)(H + 2) * u64 * 1.01;
+    const double u64 = 1.1102230246251565e-16;            // 2^-53
+    const double g_or = (double)(H + 2) * u64 * 1.01;     // the definition's own rounding, per unit of B
+    const double g_par = (double)(H / 32 + 8) * u64 * 1.01;  // warp-parallel fp64 sums
 
-    // per-token bound when no per-entry sums exist: B = sum_h |x_h| cmax_h + max|b|
-    float Btok = 0.f;
-    if (!a.absum) {
+    float xnorm = 0.f;
+    if (!F64) {  // ||x_t||_2, inflated to cover its fp32 rounding
         const uint16_t* xr = a.x + (size_t)t * H;
         float s = 0.f;
-        for (int h = lane; h < H; h += 32) s = fmaf(fabsf(bf16_bits_to_f32(xr[h])), __uint_as_float(a.cmax[h]), s);
+        for (int h = lane; h < H; h += 32) {
+            float v = bf16_bits_to_f32(xr[h]);
+            s = fmaf(v, v, s);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        // this fp32 sum of nonnegative terms (chain H/32 + 5) can be low by a
-        // relative 2 gamma at most; 1% covers it for any H here
-        Btok = s * 1.01f + (a.b ? __uint_as_float(a.cmax[H]) : 0.f) * 1.01f;
+        xnorm = sqrtf(s) * 1.001f;
     }
-    float v[NV], dl[NV];
+    double v[NV], dl[NV];
     uint32_t taken = 0;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        int e = lane + 32 * i;
+        const int e = lane + 32 * i;
         if (e < E) {
-            v[i] = a.logit[(size_t)t * E + e];
-            float B = a.absum ? a.absum[(size_t)t * E + e] * 1.01f : Btok;
-            dl[i] = B * (a.gamma32 * 1.01f) + (float)(B * g_or) + 1e-30f;
+            double B;
+            if (F64) {
+                v[i] = static_cast<const double*>(a.logit)[(size_t)t * E + e];
+                B = a.absum[(size_t)t * E + e] * (1.0 + 1e-9);
+            } else {
+                v[i] = (double)static_cast<const float*>(a.logit)[(size_t)t * E + e];
+                B = ((double)xnorm * (double)a.wnorm[e] + (a.b ? fabs((double)a.b[e]) : 0.0)) * 1.001;
+            }
+            dl[i] = B * (a.gfast + g_or) + 1e-300;
         } else {
             v[i] = -INFINITY;
-            dl[i] = 0.f;
+            dl[i] = 0.0;
             taken |= 1u << i;
         }
     }
-    // 1) top M by the fast logits
+    // 1) the best M by the fast values
     const int M = min(min(E, k + MOE_CAND_EXTRA), 32);
-    int my_e = -1;  // lane j < M holds candidate j
+    int ce = -1;
+    double cval = -INFINITY, cbnd = 0.0;
     for (int j = 0; j < M; ++j) {
-        float bv = -INFINITY;
+        double bv = -INFINITY, bd = 0.0;
         int be = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < NV; ++i)
-            if (!(taken >> i & 1u)) {
-                int e = lane + 32 * i;
-                if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
+            if (!((taken >> i) & 1u)) {
+                const int e = lane + 32 * i;
+                if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; bd = dl[i]; }
             }
-        warp_best(bv, be);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            double v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+            double d2 = __shfl_xor_sync(0xffffffffu, bd, o);
+            int e2 = __shfl_xor_sync(0xffffffffu, be, o);
+            if (v2 > bv || (v2 == bv && e2 < be)) { bv = v2; be = e2; bd = d2; }
+        }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == j) my_e = be;
+        if (lane == j) { ce = be; cval = bv; cbnd = bd; }
     }
-    // upper end of every expert outside the candidates
-    float rest = -INFINITY;
+    double rest = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-        if (!(taken >> i & 1u)) rest = fmaxf(rest, v[i] + dl[i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) rest = fmaxf(rest, __shfl_xor_sync(0xffffffffu, rest, o));
+        if (!((taken >> i) & 1u)) rest = fmax(rest, v[i] + dl[i]);
+    rest = warp_max_d(rest);
 
-    // 2) fp64 re-evaluation of the candidates (warp-parallel, bounded)
-    const double g_par = (double)(H / 32 + 8) * u64 * 1.01;
-    double cv = -INFINITY, cd = 0.0;
-    for (int j = 0; j < M; ++j) {
-        int e = __shfl_sync(0xffffffffu, my_e, j);
-        double vv, ab;
-        logit_fp64_parallel(a, t, e, vv, ab);
-        if (lane == j) { cv = vv; cd = ab * (g_par + g_or) + 1e-300; }
-    }
-    // 3) sorted position of each candidate by (cv desc, e asc)
-    int rank = 0;
-    for (int j = 0; j < M; ++j) {
-        double oj = __shfl_sync(0xffffffffu, cv, j);
-        int ej = __shfl_sync(0xffffffffu, my_e, j);
-        if (lane < M && (oj > cv || (oj == cv && ej < my_e))) ++rank;
-    }
-    // gather candidates into sorted order: lane r receives position r
-    int src = 0;
-    for (int j = 0; j < M; ++j) {
-        int rj = __shfl_sync(0xffffffffu, rank, j);
-        if (rj == lane) src = j;
-    }
-    double sv = __shfl_sync(0xffffffffu, cv, src);
-    double sd = __shfl_sync(0xffffffffu, cd, src);
-    int se = __shfl_sync(0xffffffffu, my_e, src);
-    double nv = __shfl_down_sync(0xffffffffu, sv, 1);
-    double nd = __shfl_down_sync(0xffffffffu, sd, 1);
-    // 4) certification: positions r < k are strictly separated from r + 1
-    //    (when it exists) and the k-th chosen clears every non-candidate
-    bool ok = true;
-    if (lane < k && lane + 1 < M) ok = (sv - sd) > (nv + nd);
-    if (lane == k - 1) ok = ok && ((sv - sd) > (double)rest || rest == -INFINITY);
-    const bool certified = __all_sync(0xffffffffu, ok);
-
-    if (certified) {
-        double v0 = __shfl_sync(0xffffffffu, sv, 0);
-        double z = (lane < k) ? exp(sv - v0) : 0.0;
-        double zs = warp_sum_d(z);
-        if (lane < k) {
-            a.idx[(size_t)t * k + lane] = se;
-            a.w[(size_t)t * k + lane] = (float)(z / zs);
-        }
+    // 2) certified on the fast values?
+    if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
+        write_topk(a, t, cval, ce);
         return;
     }
-
-    // 5) exact path: every expert whose upper end reaches theta, the lowest
-    //    lower end among the chosen k, is evaluated by the definition
-    double th = (lane < k) ? (sv - sd) : INFINITY;
+    // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
+    if (!F64) {
+        for (int base = 0; base < M; base += 16) {
+            int ej[16];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) th = fmin(th, __shfl_xor_sync(0xffffffffu, th, o));
-    int* ce = s_ce[wid];
+            for (int j = 0; j < 16; ++j) ej[j] = __shfl_sync(0xffffffffu, ce, min(base + j, 31));
+            double acc[16], ab[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = ab[j] = 0.0;
+            const uint16_t* xr = a.x + (size_t)t * H;
+            for (int h = lane; h < H; h += 32) {
+                const double xd = bf16_bits_to_f32(xr[h]);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (base + j < M) {
+                        const double p = xd * (double)__ldg(a.W + (size_t)ej[j] * H + h);
+                        acc[j] += p;
+                        ab[j] += fabs(p);
+                    }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (base + j < M) {
+                    const double s = warp_sum_d(acc[j]), sa = warp_sum_d(ab[j]);
+                    const double bb = a.b ? (double)a.b[ej[j]] : 0.0;
+                    if (lane == base + j) {
+                        cval = s + bb;
+                        cbnd = (sa + fabs(bb)) * (1.0 + 1e-9) * (g_par + g_or) + 1e-300;
+                    }
+                }
+            }
+        }
+        if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
+            write_topk(a, t, cval, ce);
+            return;
+        }
+    }
+    // 4) exact: every expert whose upper end reaches theta (the lowest lower
+    //    end among the k best) is evaluated by the definition itself
+    const double th = warp_min_d(lane < k ? cval - cbnd : INFINITY);
+    int* cs = s_ce[wid];
     double* cvs = s_cv[wid];
     int nc = 0;
     for (int i = 0; i < NV; ++i) {
-        int e = lane + 32 * i;
-        // the candidates of step 1 (marked taken) are always kept
-        bool in = (e < E) && (((taken >> i) & 1u) || (double)v[i] + (double)dl[i] >= th);
-        unsigned m = __ballot_sync(0xffffffffu, in);
-        if (in) ce[nc + __popc(m & ((1u << lane) - 1))] = e;
+        const int e = lane + 32 * i;
+        // the step-1 candidates (marked taken) are always kept
+        const bool in = (e < E) && ((((taken >> i) & 1u) != 0) || v[i] + dl[i] >= th);
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        if (in) cs[nc + __popc(m & ((1u << lane) - 1))] = e;
         nc += __popc(m);
     }
     __syncwarp();
-    for (int c = lane; c < nc; c += 32) cvs[c] = logit_fp64_exact(a, t, ce[c]);
+    for (int c = lane; c < nc; c += 32) cvs[c] = logit_fp64_exact(a, t, cs[c]);
     __syncwarp();
-    // select k from the exact values, ties to the lower index
-    double l0 = 0.0, z = 0.0;
+    double l0 = 0.0, z = 0.0, mine = 0.0;
     for (int j = 0; j < k; ++j) {
         double bv = -INFINITY;
         int be = 0x7fffffff, bc = -1;
         for (int c = lane; c < nc; c += 32)
-            if (ce[c] >= 0 && (cvs[c] > bv || (cvs[c] == bv && ce[c] < be))) { bv = cvs[c]; be = ce[c]; bc = c; }
-        int bcw = bc;
-        double bvw = bv;
-        int bew = be;
+            if (cs[c] >= 0 && (cvs[c] > bv || (cvs[c] == bv && cs[c] < be))) { bv = cvs[c]; be = cs[c]; bc = c; }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            double v2 = __shfl_xor_sync(0xffffffffu, bvw, o);
-            int e2 = __shfl_xor_sync(0xffffffffu, bew, o);
-            int c2 = __shfl_xor_sync(0xffffffffu, bcw, o);
-            if (v2 > bvw || (v2 == bvw && e2 < bew)) { bvw = v2; bew = e2; bcw = c2; }
+            double v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+            int e2 = __shfl_xor_sync(0xffffffffu, be, o);
+            int c2 = __shfl_xor_sync(0xffffffffu, bc, o);
+            if (v2 > bv || (v2 == bv && e2 < be)) { bv = v2; be = e2; bc = c2; }
         }
         __syncwarp();
         if (lane == 0) {
-            ce[bcw] = -1;  // remove from the pool
-            a.idx[(size_t)t * k + j] = bew;
+            cs[bc] = -1;  // taken
+            a.idx[(size_t)t * k + j] = be;
         }
         __syncwarp();
-        if (j == 0) l0 = bvw;
-        double zz = exp(bvw - l0);
+        if (j == 0) l0 = bv;
+        const double zz = exp(bv - l0);
         z += zz;
-        if (lane == j) cd = zz;  // reuse: lane j keeps its numerator
+        if (lane == j) mine = zz;
     }
-    if (lane < k) a.w[(size_t)t * k + lane] = (float)(cd / z);
+    if (lane < k) a.w[(size_t)t * k + lane] = (float)(mine / z);
     if (lane == 0 && a.n_rechecked) atomicAdd(a.n_rechecked, 1);
 }

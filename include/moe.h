@@ -184,6 +184,11 @@ const char* moe_strerror(int code);
 int moe_set_stage_events(void* const* events, int n);
 uint64_t moe_launch_count(void);
 
+/* Diagnostic companion of MOE_ERR_TIMEOUT: after synchronising `stream`,
+ * returns and clears where the first bounded device wait gave up
+ * (site * 1000000 + CTA * 1000 + unit, 0 = none); negative on CUDA failure. */
+int moe_timeout_site(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

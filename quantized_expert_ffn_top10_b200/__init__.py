@@ -42,7 +42,7 @@ MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T = 8, 8192
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",
            "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
-           "moe_set_stage_events", "moe_launch_count")
+           "moe_set_stage_events", "moe_launch_count", "moe_timeout_site")
 
 
 class RouteOut(ctypes.Structure):
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.moe_set_stage_events.argtypes = [P, i32]
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_launch_count.argtypes = []
+        L.moe_timeout_site.restype = i32
+        L.moe_timeout_site.argtypes = [P]
         _lib = L
     return _lib
 
@@ -195,3 +197,7 @@ def moe_set_stage_events(events) -> int:
 
 def moe_launch_count() -> int:
     return int(lib().moe_launch_count())
+
+
+def moe_timeout_site(stream=None) -> int:
+    return int(lib().moe_timeout_site(_stream(stream)))

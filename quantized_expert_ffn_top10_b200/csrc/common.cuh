@@ -20,6 +20,14 @@ __device__ int g_moe_status;
 
 __device__ __forceinline__ void moe_set_status(int code) { atomicCAS(&g_moe_status, 0, code); }
 
+// Where the first bounded wait gave up (0 = nowhere): site * 1000000 + CTA * 1000 + detail.
+__device__ int g_moe_where;
+
+__device__ __forceinline__ void moe_note_timeout(int site, int detail) {
+    moe_set_status(MOE_ERR_TIMEOUT);
+    atomicCAS(&g_moe_where, 0, site * 1000000 + (int)(blockIdx.x % 1000) * 1000 + min(detail, 999));
+}
+
 // Upper bound on iterations of any spin wait (each iteration sleeps ~0.1-1 us
 // after the first few); about 2 s in total.  On expiry the waiter latches
 // MOE_ERR_TIMEOUT and gives up instead of hanging the GPU.
@@ -81,12 +89,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and latches MOE_ERR_TIMEOUT) if it did not complete within the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site = 9, int detail = 0) {
     for (uint32_t it = 0; it < MOE_SPIN_LIMIT; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (it > 64) __nanosleep(64);
     }
-    moe_set_status(MOE_ERR_TIMEOUT);
+    moe_note_timeout(site, detail);
     return false;
 }
 

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_fused.cuh"
 #include "perm.cuh"
 #include "prefill.cuh"
 #include "router.cuh"
@@ -59,6 +60,8 @@ std::mutex g_mu;
 std::vector<cudaEvent_t> g_stage_ev;  // measurement hook, see moe_set_stage_events
 std::atomic<uint64_t> g_launches{0};
 uint64_t g_init_mask[4] = {0, 0, 0, 0};  // devices whose kernel attributes are set
+int g_df_grid[256];                     // fused-decode grid (one CTA per SM) per device, 0 = unusable
+constexpr int kDfMaxH = 2560;           // largest H the fused decode kernel stages
 
 inline void stage(int i, cudaStream_t st) {
     std::lock_guard<std::mutex> g(g_mu);
@@ -185,6 +188,30 @@ bool tmap_codes(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_b
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// codes of one matrix, 16-row boxes of 128 bytes with 128-byte swizzle (fused decode staging)
+bool tmap_codes_sw(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t n_slots,
+                   int64_t slot_bytes) {
+    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_slots};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)slot_bytes};
+    cuuint32_t box[3] = {128, 16, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 scales of one matrix [n_slots][rows][K/32], box (kb/32) x 16 x 1
+bool tmap_scales(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t K, int64_t n_slots, int64_t slot_bytes,
+                 int kb) {
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 32), (cuuint64_t)rows, (cuuint64_t)n_slots};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 32 * 2), (cuuint64_t)slot_bytes};
+    cuuint32_t box[3] = {(cuuint32_t)(kb / 32), 16, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -208,6 +235,15 @@ int ensure_init() {
     chk(set_smem(k_prefill_gemm<0, 4, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 2, 2>, PfCfg<0>::SMEM));
     chk(set_smem(k_prefill_gemm<0, 2, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 4, 2>, PfCfg<0>::SMEM));
     chk(set_smem(k_prefill_gemm<1, 4, 4>, PfCfg<1>::SMEM)); chk(set_smem(k_prefill_gemm<1, 2, 2>, PfCfg<1>::SMEM));
+    const int dfs = df_smem_bytes(kDfMaxH);
+    chk(set_smem(k_decode_fused<4, 4, 4>, dfs)); chk(set_smem(k_decode_fused<2, 2, 4>, dfs));
+    chk(set_smem(k_decode_fused<4, 4, 2>, dfs)); chk(set_smem(k_decode_fused<2, 2, 2>, dfs));
+    chk(set_smem(k_decode_fused<2, 4, 4>, dfs)); chk(set_smem(k_decode_fused<4, 2, 4>, dfs));
+    chk(set_smem(k_decode_fused<2, 4, 2>, dfs)); chk(set_smem(k_decode_fused<4, 2, 2>, dfs));
+    int nsm = 0, per = 0;
+    chk(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4, 4>, DF_THREADS, dfs));
+    g_df_grid[dev] = (per >= 1) ? nsm : 0;
     if (e != cudaSuccess || !encoder()) return MOE_ERR_CUDA;
     g_init_mask[dev >> 6] |= 1ull << (dev & 63);
     return MOE_OK;
@@ -279,7 +315,94 @@ void launch_down(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
     k_dec_down<BD><<<dim3((a.H + 31) / 32, umax), 32 * DEC_DN_WARPS, smem, st>>>(a);
 }
 
+// Shapes the fused decode kernel stages: gate/up K-chunks of min(H, 1024)
+// with 128-byte code rows per chunk and 16-byte scale rows; down rows of
+// 128-byte multiples; everything within one ring slot and the smem plan.
+bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || g_df_grid[dev] < 1) return false;
+    const int H = d->H, I = d->I, chunk = std::min(H, 1024);
+    if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH) return false;
+    if (H % chunk || chunk % 256 || I % 256) return false;
+    if ((chunk * d->bits_gate / 8) % 128 || (chunk * d->bits_up / 8) % 128 || (I * d->bits_down / 8) % 128) return false;
+    if ((chunk * d->bits_gate / 8 / 128 + chunk * d->bits_up / 8 / 128) * 2048 + 2 * 16 * (chunk / 32) * 2 > DF_SLOT)
+        return false;
+    if ((I * d->bits_down / 8 / 128) * 2048 + 16 * (I / 32) * 2 > DF_SLOT) return false;
+    return true;
+}
+
+template <int BG, int BU, int BD>
+cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(DF_THREADS);
+    cfg.dynamicSmemBytes = df_smem_bytes(kDfMaxH);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;  // all CTAs co-resident: the grid barriers rely on it
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<BG, BU, BD>, tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], a);
+}
+
+int run_decode_fused(const LayerCall& c) {
+    const moe_arena_desc* d = c.d;
+    const int H = d->H, I = d->I;
+    const Ws L = ws_layout(c.T, c.E, c.k, H, I);
+    const moe_route_out* ro = c.ro;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    DecodeFusedArgs a{};
+    a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = d->n_slots; a.slot_bytes = d->slot_bytes;
+    for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
+    a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.residual;
+    a.bits_g = d->bits_gate; a.bits_u = d->bits_up; a.bits_d = d->bits_down;
+    a.chunk = std::min(H, 1024);
+    a.x = c.x; a.W = c.W; a.b = c.b; a.out = c.out; a.hist = c.hist;
+    a.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
+    a.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
+    a.offsets = (ro && ro->expert_offsets) ? ro->expert_offsets : reinterpret_cast<int32_t*>(c.ws + L.offsets);
+    a.perm = (ro && ro->perm) ? ro->perm : reinterpret_cast<int32_t*>(c.ws + L.perm);
+    a.nrechk = (ro && ro->n_rechecked) ? ro->n_rechecked : reinterpret_cast<int32_t*>(c.ws + L.nrechk);
+    a.logit = reinterpret_cast<double*>(c.ws + L.logit);
+    a.absum = reinterpret_cast<double*>(c.ws + L.absum);
+    a.hB = reinterpret_cast<uint16_t*>(c.ws + L.h);
+    a.hC = reinterpret_cast<float*>(c.ws + L.y);
+    a.bar = reinterpret_cast<unsigned int*>(c.ws + L.meta + 8);
+    CUtensorMap tm[6];
+    const int64_t ns = d->n_slots, sb = d->slot_bytes;
+    const int chunk = a.chunk;
+    if (!tmap_codes_sw(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8, ns, sb) ||
+        !tmap_codes_sw(&tm[1], c.arena + d->off_codes[1], I, (int64_t)H * d->bits_up / 8, ns, sb) ||
+        !tmap_codes_sw(&tm[2], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb) ||
+        !tmap_scales(&tm[3], c.arena + d->off_scales[0], I, H, ns, sb, chunk) ||
+        !tmap_scales(&tm[4], c.arena + d->off_scales[1], I, H, ns, sb, chunk) ||
+        !tmap_scales(&tm[5], c.arena + d->off_scales[2], H, I, ns, sb, I))
+        return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(a.bar, 0, 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    stage(0, c.st);
+    const int grid = g_df_grid[dev];
+    const int key = d->bits_gate * 100 + d->bits_up * 10 + d->bits_down;
+    cudaError_t e;
+    switch (key) {
+        case 444: e = launch_fused<4, 4, 4>(tm, a, grid, c.st); break;
+        case 224: e = launch_fused<2, 2, 4>(tm, a, grid, c.st); break;
+        case 442: e = launch_fused<4, 4, 2>(tm, a, grid, c.st); break;
+        case 222: e = launch_fused<2, 2, 2>(tm, a, grid, c.st); break;
+        case 244: e = launch_fused<2, 4, 4>(tm, a, grid, c.st); break;
+        case 424: e = launch_fused<4, 2, 4>(tm, a, grid, c.st); break;
+        case 242: e = launch_fused<2, 4, 2>(tm, a, grid, c.st); break;
+        default: e = launch_fused<4, 2, 2>(tm, a, grid, c.st); break;
+    }
+    for (int i = 1; i < 5; ++i) stage(i, c.st);  // one kernel: the stages collapse onto its end
+    count(1);
+    return e == cudaSuccess ? cuda_rc(cudaGetLastError()) : MOE_ERR_CUDA;
+}
+
 int run_decode(const LayerCall& c) {
+    if (fused_decode_ok(c.d, c.T, c.E, c.k)) return run_decode_fused(c);
     const moe_arena_desc* d = c.d;
     const Ws L = ws_layout(c.T, c.E, c.k, d->H, d->I);
     Routed r;
@@ -461,6 +584,14 @@ int moe_set_stage_events(void* const* events, int n) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_timeout_site(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_moe_where, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_moe_where, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
 
 const char* moe_strerror(int code) {
     switch (code) {

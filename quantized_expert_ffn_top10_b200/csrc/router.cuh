@@ -242,25 +242,24 @@ __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ void write_topk(const TopkArgs& a, int t, double cval, int ce) {
+__device__ __forceinline__ void write_topk(int k, double cval, int ce, int32_t* idx_out, float* w_out) {
     const int lane = threadIdx.x & 31;
     const double v0 = __shfl_sync(0xffffffffu, cval, 0);
-    const double z = (lane < a.k) ? exp(cval - v0) : 0.0;
+    const double z = (lane < k) ? exp(cval - v0) : 0.0;
     const double zs = warp_sum_d(z);
-    if (lane < a.k) {
-        a.idx[(size_t)t * a.k + lane] = ce;
-        a.w[(size_t)t * a.k + lane] = (float)(z / zs);
+    if (lane < k) {
+        idx_out[lane] = ce;
+        w_out[lane] = (float)(z / zs);
     }
 }
 
-// One warp per token; lanes hold the fast logits of experts e = lane + 32 i.
+// Top-k of token t by one warp; lanes hold the fast logits of experts
+// e = lane + 32 i.  Results go to idx_out[0..k) / w_out[0..k); cs / cvs are
+// per-warp scratch of MOE_MAX_E entries for the exact path.
 template <bool F64>
-__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
-    __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
-    __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int t = blockIdx.x * MOE_TOPK_WARPS + wid;
-    if (t >= a.T) return;
+__device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* idx_out, float* w_out, int* cs,
+                                           double* cvs, int32_t* nrechk) {
+    const int lane = threadIdx.x & 31;
     const int E = a.E, k = a.k, H = a.H;
     constexpr int NV = MOE_MAX_E / 32;
     const double u64 = 1.1102230246251565e-16;            // 2^-53
@@ -331,7 +330,7 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
 
     // 2) certified on the fast values?
     if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
-        write_topk(a, t, cval, ce);
+        write_topk(k, cval, ce, idx_out, w_out);
         return;
     }
     // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
@@ -367,15 +366,13 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
             }
         }
         if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
-            write_topk(a, t, cval, ce);
+            write_topk(k, cval, ce, idx_out, w_out);
             return;
         }
     }
     // 4) exact: every expert whose upper end reaches theta (the lowest lower
     //    end among the k best) is evaluated by the definition itself
     const double th = warp_min_d(lane < k ? cval - cbnd : INFINITY);
-    int* cs = s_ce[wid];
-    double* cvs = s_cv[wid];
     int nc = 0;
     for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
@@ -404,7 +401,7 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
         __syncwarp();
         if (lane == 0) {
             cs[bc] = -1;  // taken
-            a.idx[(size_t)t * k + j] = be;
+            idx_out[j] = be;
         }
         __syncwarp();
         if (j == 0) l0 = bv;
@@ -412,6 +409,17 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
         z += zz;
         if (lane == j) mine = zz;
     }
-    if (lane < k) a.w[(size_t)t * k + lane] = (float)(mine / z);
-    if (lane == 0 && a.n_rechecked) atomicAdd(a.n_rechecked, 1);
+    if (lane < k) w_out[lane] = (float)(mine / z);
+    if (lane == 0 && nrechk) atomicAdd(nrechk, 1);
+}
+
+// One warp per token.
+template <bool F64>
+__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
+    __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
+    __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
+    const int wid = threadIdx.x >> 5;
+    const int t = blockIdx.x * MOE_TOPK_WARPS + wid;
+    if (t >= a.T) return;
+    topk_token<F64>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
 }

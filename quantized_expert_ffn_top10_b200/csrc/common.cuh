@@ -90,10 +90,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and latches MOE_ERR_TIMEOUT) if it did not complete within the limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site = 9, int detail = 0) {
-    for (uint32_t it = 0; it < MOE_SPIN_LIMIT; ++it) {
+    // try_wait suspends the thread until the phase completes or a short
+    // hardware time limit passes, so the loop wakes promptly without sleeping
+    for (uint32_t it = 0; it < MOE_SPIN_LIMIT; ++it)
         if (mbar_try_wait(bar, parity)) return true;
-        if (it > 64) __nanosleep(64);
-    }
     moe_note_timeout(site, detail);
     return false;
 }

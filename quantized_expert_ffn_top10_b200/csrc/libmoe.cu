@@ -123,7 +123,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
         k_router_gemv<<<(E + 7) / 8, 256, 0, st>>>(x, T, H, W, b, E, logit, absum);
         ta.absum = absum;
         ta.gfast = gamma_n(H / 32 + 6, 1.1102230246251565e-16);
-        k_topk<true><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+        k_topk<1><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     } else {
         float* wnorm = reinterpret_cast<float*>(ws + L.cmax);
         float* logit = reinterpret_cast<float*>(ws + L.logit);
@@ -131,7 +131,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
         k_router_gemm<<<dim3((E + RG_BN - 1) / RG_BN, (T + RG_BM - 1) / RG_BM), 256, 0, st>>>(x, T, H, W, b, E, logit);
         ta.wnorm = wnorm;
         ta.gfast = gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);
-        k_topk<false><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+        k_topk<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     }
     PermArgs pa{};
     pa.idx = idx; pa.P = P; pa.E = E; pa.nchunks = (P + PERM_CHUNK - 1) / PERM_CHUNK;
@@ -321,13 +321,15 @@ void launch_down(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
 bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || g_df_grid[dev] < 1) return false;
-    const int H = d->H, I = d->I, chunk = std::min(H, 1024);
-    if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH) return false;
-    if (H % chunk || chunk % 256 || I % 256) return false;
-    if ((chunk * d->bits_gate / 8) % 128 || (chunk * d->bits_up / 8) % 128 || (I * d->bits_down / 8) % 128) return false;
-    if ((chunk * d->bits_gate / 8 / 128 + chunk * d->bits_up / 8 / 128) * 2048 + 2 * 16 * (chunk / 32) * 2 > DF_SLOT)
+    const int H = d->H, I = d->I;
+    if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH || H % DF_CHUNK || I % 256) return false;
+    if ((I * d->bits_down / 8) % 128) return false;
+    // one phase-D unit: W_d rows, scales, h and half-block sums of up to T pairs
+    const int hs = std::min(T, DF_HSTAGE);
+    if ((I * d->bits_down / 8 / 128) * 2048 + 16 * (I / 32) * 2 + hs * I * 2 + hs * (I / 16) * 4 > DF_SLOT) return false;
+    if ((DF_CHUNK * d->bits_gate / 8 / 128 + DF_CHUNK * d->bits_up / 8 / 128) * 2048 + 2 * 16 * (DF_CHUNK / 32) * 2 >
+        DF_SLOT)
         return false;
-    if ((I * d->bits_down / 8 / 128) * 2048 + 16 * (I / 32) * 2 > DF_SLOT) return false;
     return true;
 }
 
@@ -358,7 +360,6 @@ int run_decode_fused(const LayerCall& c) {
     for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
     a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.residual;
     a.bits_g = d->bits_gate; a.bits_u = d->bits_up; a.bits_d = d->bits_down;
-    a.chunk = std::min(H, 1024);
     a.x = c.x; a.W = c.W; a.b = c.b; a.out = c.out; a.hist = c.hist;
     a.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
     a.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
@@ -367,12 +368,13 @@ int run_decode_fused(const LayerCall& c) {
     a.nrechk = (ro && ro->n_rechecked) ? ro->n_rechecked : reinterpret_cast<int32_t*>(c.ws + L.nrechk);
     a.logit = reinterpret_cast<double*>(c.ws + L.logit);
     a.absum = reinterpret_cast<double*>(c.ws + L.absum);
+    a.wnorm = reinterpret_cast<float*>(c.ws + L.cmax);
     a.hB = reinterpret_cast<uint16_t*>(c.ws + L.h);
     a.hC = reinterpret_cast<float*>(c.ws + L.y);
     a.bar = reinterpret_cast<unsigned int*>(c.ws + L.meta + 8);
     CUtensorMap tm[6];
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
-    const int chunk = a.chunk;
+    const int chunk = DF_CHUNK;
     if (!tmap_codes_sw(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8, ns, sb) ||
         !tmap_codes_sw(&tm[1], c.arena + d->off_codes[1], I, (int64_t)H * d->bits_up / 8, ns, sb) ||
         !tmap_codes_sw(&tm[2], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb) ||

@@ -179,6 +179,7 @@ struct TopkArgs {
     const float* b;         // [E] or null
     const void* logit;      // [T][E]: double (decode) or float (prefill) fast logits
     const double* absum;    // decode: [T][E] sums of |x W| + |b|
+    const float* xnorm;     // [T] upper bounds of ||x_t||_2, or null (computed here)
     const float* wnorm;     // prefill: [E] upper bounds of ||W[e]||_2
     int32_t* idx;           // [T][k]
     float* w;               // [T][k]
@@ -245,20 +246,26 @@ __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int
 __device__ __forceinline__ void write_topk(int k, double cval, int ce, int32_t* idx_out, float* w_out) {
     const int lane = threadIdx.x & 31;
     const double v0 = __shfl_sync(0xffffffffu, cval, 0);
-    const double z = (lane < k) ? exp(cval - v0) : 0.0;
-    const double zs = warp_sum_d(z);
+    const float z = (lane < k) ? expf((float)(cval - v0)) : 0.f;  // differences are small: fp32 exp suffices
+    float zs = z;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
     if (lane < k) {
         idx_out[lane] = ce;
-        w_out[lane] = (float)(z / zs);
+        w_out[lane] = z / zs;
     }
 }
 
 // Top-k of token t by one warp; lanes hold the fast logits of experts
 // e = lane + 32 i.  Results go to idx_out[0..k) / w_out[0..k); cs / cvs are
 // per-warp scratch of MOE_MAX_E entries for the exact path.
-template <bool F64>
+// MODE 0: fp32 logits, bound from norms (prefill); 1: fp64 logits with
+// per-entry sums of |x W| (decode kernels); 2: fp64 logits, bound from norms
+// (fused decode, whose router runs on the fp64 tensor cores).
+template <int MODE>
 __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* idx_out, float* w_out, int* cs,
                                            double* cvs, int32_t* nrechk) {
+    constexpr bool F64 = MODE != 0;
     const int lane = threadIdx.x & 31;
     const int E = a.E, k = a.k, H = a.H;
     constexpr int NV = MOE_MAX_E / 32;
@@ -267,60 +274,88 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     const double g_par = (double)(H / 32 + 8) * u64 * 1.01;  // warp-parallel fp64 sums
 
     float xnorm = 0.f;
-    if (!F64) {  // ||x_t||_2, inflated to cover its fp32 rounding
-        const uint16_t* xr = a.x + (size_t)t * H;
-        float s = 0.f;
-        for (int h = lane; h < H; h += 32) {
-            float v = bf16_bits_to_f32(xr[h]);
-            s = fmaf(v, v, s);
-        }
+    if (MODE != 1) {  // ||x_t||_2, inflated to cover its fp32 rounding
+        if (a.xnorm) {
+            xnorm = a.xnorm[t];
+        } else {
+            const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)t * H);
+            float s = 0.f;
+            for (int i = lane; i < H / 8; i += 32) {
+                const uint4 r = __ldg(xr + i);
+                const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        xnorm = sqrtf(s) * 1.001f;
+                for (int z = 0; z < 4; ++z) {
+                    const float lo = __uint_as_float(wd[z] << 16), hi = __uint_as_float(wd[z] & 0xffff0000u);
+                    s = fmaf(lo, lo, fmaf(hi, hi, s));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            xnorm = sqrtf(s) * 1.001f;
+        }
     }
     double v[NV], dl[NV];
+    uint32_t key[NV];  // order-preserving 32-bit keys of the values rounded to fp32
     uint32_t taken = 0;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
             double B;
+            float f;
             if (F64) {
                 v[i] = static_cast<const double*>(a.logit)[(size_t)t * E + e];
-                B = a.absum[(size_t)t * E + e] * (1.0 + 1e-9);
+                f = (float)v[i];
             } else {
-                v[i] = (double)static_cast<const float*>(a.logit)[(size_t)t * E + e];
-                B = ((double)xnorm * (double)a.wnorm[e] + (a.b ? fabs((double)a.b[e]) : 0.0)) * 1.001;
+                f = static_cast<const float*>(a.logit)[(size_t)t * E + e];
+                v[i] = (double)f;
             }
+            if (MODE == 1) B = a.absum[(size_t)t * E + e] * (1.0 + 1e-9);
+            else B = ((double)xnorm * (double)a.wnorm[e] + (a.b ? fabs((double)a.b[e]) : 0.0)) * 1.001;
             dl[i] = B * (a.gfast + g_or) + 1e-300;
+            const uint32_t u = __float_as_uint(f);
+            key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         } else {
             v[i] = -INFINITY;
             dl[i] = 0.0;
+            key[i] = 0;
             taken |= 1u << i;
         }
     }
-    // 1) the best M by the fast values
+    // 1) M candidates, picked by the 32-bit keys with warp reductions; a
+    //    candidate set that misses a member of the true top k only fails the
+    //    certification below.
     const int M = min(min(E, k + MOE_CAND_EXTRA), 32);
     int ce = -1;
     double cval = -INFINITY, cbnd = 0.0;
-    for (int j = 0; j < M; ++j) {
-        double bv = -INFINITY, bd = 0.0;
-        int be = 0x7fffffff;
+    uint32_t lkey = 0;
+    int li = -1;
+    auto rescan = [&]() {  // this lane's best untaken entry (lowest index on equal keys)
+        lkey = 0;
+        li = -1;
 #pragma unroll
         for (int i = 0; i < NV; ++i)
-            if (!((taken >> i) & 1u)) {
-                const int e = lane + 32 * i;
-                if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; bd = dl[i]; }
-            }
+            if (!((taken >> i) & 1u) && (li < 0 || key[i] > lkey)) { lkey = key[i]; li = i; }
+    };
+    rescan();
+    for (int j = 0; j < M; ++j) {
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, lkey);
+        const uint32_t me =
+            __reduce_min_sync(0xffffffffu, (li >= 0 && lkey == mk) ? (uint32_t)(lane + 32 * li) : 0xffffffffu);
+        const int owner = (int)(me & 31u);
+        double lv = 0.0, ld = 0.0;
+        if (lane == owner) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            double v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-            double d2 = __shfl_xor_sync(0xffffffffu, bd, o);
-            int e2 = __shfl_xor_sync(0xffffffffu, be, o);
-            if (v2 > bv || (v2 == bv && e2 < be)) { bv = v2; be = e2; bd = d2; }
+            for (int i = 0; i < NV; ++i)
+                if (i == li) { lv = v[i]; ld = dl[i]; }
         }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == j) { ce = be; cval = bv; cbnd = bd; }
+        const double bv = __shfl_sync(0xffffffffu, lv, owner);
+        const double bd = __shfl_sync(0xffffffffu, ld, owner);
+        if (lane == j) { ce = (int)me; cval = bv; cbnd = bd; }
+        if (lane == owner) {
+            taken |= 1u << li;
+            rescan();
+        }
     }
     double rest = -INFINITY;
 #pragma unroll
@@ -334,7 +369,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         return;
     }
     // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
-    if (!F64) {
+    if (MODE == 0) {
         for (int base = 0; base < M; base += 16) {
             int ej[16];
 #pragma unroll
@@ -405,7 +440,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         }
         __syncwarp();
         if (j == 0) l0 = bv;
-        const double zz = exp(bv - l0);
+        const double zz = (double)expf((float)(bv - l0));
         z += zz;
         if (lane == j) mine = zz;
     }
@@ -414,12 +449,12 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
 }
 
 // One warp per token.
-template <bool F64>
+template <int MODE>
 __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk(TopkArgs a) {
     __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
     __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
     const int wid = threadIdx.x >> 5;
     const int t = blockIdx.x * MOE_TOPK_WARPS + wid;
     if (t >= a.T) return;
-    topk_token<F64>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
+    topk_token<MODE>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
 }

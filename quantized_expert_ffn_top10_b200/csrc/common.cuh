@@ -77,22 +77,24 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// Waits up to about suspend_ns for the phase with this parity to complete;
+// the warp is suspended meanwhile (no issue slots used) and woken when it does.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns = 20000) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
         : "memory");
     return ok != 0;
 }
 
+#define MOE_WAIT_ROUNDS (1u << 17)  // x 20 us suspend hint: the bound on any mbarrier wait
+
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and latches MOE_ERR_TIMEOUT) if it did not complete within the limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site = 9, int detail = 0) {
-    // try_wait suspends the thread until the phase completes or a short
-    // hardware time limit passes, so the loop wakes promptly without sleeping
-    for (uint32_t it = 0; it < MOE_SPIN_LIMIT; ++it)
+    for (uint32_t it = 0; it < MOE_WAIT_ROUNDS; ++it)
         if (mbar_try_wait(bar, parity)) return true;
     moe_note_timeout(site, detail);
     return false;

@@ -494,15 +494,32 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     const bool consumer = warp >= 1 && warp <= DF_GROUPS * DF_GW;
     float* gpart = reinterpret_cast<float*>(ypair + DF_MAXP * DF_FT);  // [group][warp][lane][8] partial sums
 
-    if (alive && ft0 < H)  // W_d rows of phase D into L2 while gate/up streams from HBM
-        for (int ft = ft0; ft < H; ft += G * DF_FT)
-            for (int ui = tid; ui < nuq; ui += DF_THREADS) {
-                const int64_t sl = a.slot_table[(int64_t)a.layer * E + rt->u_e[ui]];
-                if (sl < 0 || sl >= a.n_slots) continue;
-                const uint8_t* base = a.arena + sl * a.slot_bytes;
-                prefetch_l2(base + a.off_codes[2] + (int64_t)ft * rowb_d, (uint32_t)(DF_FT * rowb_d));
-                prefetch_l2(base + a.off_scales[2] + (int64_t)ft * (I / 32) * 2, (uint32_t)(DF_FT * (I / 32) * 2));
-            }
+    // Everything this CTA will read in C and D goes to L2 at once: HBM then
+    // streams at full rate whatever the shared-memory ring can hold, and the
+    // ring refills from L2.  Gate/up tiles first (16 contiguous rows each),
+    // then the W_d rows of this CTA's features for every selected expert.
+    if (alive) {
+        const int rowb_g = H * BG / 8, rowb_u = H * BU / 8;
+        for (int lt = tid; lt < nloc; lt += DF_THREADS) {
+            const int gt = r0 + lt, ui = gt / tiles_per_e, r16 = gt % tiles_per_e;
+            const int64_t sl = a.slot_table[(int64_t)a.layer * E + rt->u_e[ui]];
+            if (sl < 0 || sl >= a.n_slots) continue;
+            const uint8_t* base = a.arena + sl * a.slot_bytes;
+            prefetch_l2(base + a.off_codes[0] + (int64_t)r16 * 16 * rowb_g, (uint32_t)(16 * rowb_g));
+            prefetch_l2(base + a.off_codes[1] + (int64_t)r16 * 16 * rowb_u, (uint32_t)(16 * rowb_u));
+            prefetch_l2(base + a.off_scales[0] + (int64_t)r16 * 16 * (H / 16), (uint32_t)(16 * (H / 16)));
+            prefetch_l2(base + a.off_scales[1] + (int64_t)r16 * 16 * (H / 16), (uint32_t)(16 * (H / 16)));
+        }
+        if (ft0 < H)
+            for (int ft = ft0; ft < H; ft += G * DF_FT)
+                for (int ui = tid; ui < nuq; ui += DF_THREADS) {
+                    const int64_t sl = a.slot_table[(int64_t)a.layer * E + rt->u_e[ui]];
+                    if (sl < 0 || sl >= a.n_slots) continue;
+                    const uint8_t* base = a.arena + sl * a.slot_bytes;
+                    prefetch_l2(base + a.off_codes[2] + (int64_t)ft * rowb_d, (uint32_t)(DF_FT * rowb_d));
+                    prefetch_l2(base + a.off_scales[2] + (int64_t)ft * (I / 32) * 2, (uint32_t)(DF_FT * (I / 32) * 2));
+                }
+    }
 
     const bool producer = warp >= DF_WARPS - DF_GROUPS;  // warps 13..15 feed groups 0..2
     if (producer) {

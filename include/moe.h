@@ -50,6 +50,7 @@ extern "C" {
 #define MOE_ERR_CUDA (-5)     /* a CUDA launch or query failed                  */
 #define MOE_ERR_SLOT (-6)     /* a selected expert had slot -1 or >= n_slots    */
 #define MOE_ERR_TIMEOUT (-7)  /* a bounded device-side wait expired             */
+#define MOE_ERR_STATIC (-8)   /* size beyond moe_route_static's fixed scratch    */
 
 #define MOE_MAX_E 512         /* experts per layer                              */
 #define MOE_MAX_TOPK 32
@@ -115,6 +116,29 @@ size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I);
 int moe_route(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias,
               int E, int top_k, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
               int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_route without a caller workspace: the same router and grouping kernels,
+ * with their scratch in a fixed device array inside libmoe.so
+ * (MOE_ROUTE_STATIC_BYTES per device, located once per device with
+ * cudaGetSymbolAddress).  No page of the method has a counterpart: it is a
+ * serving convenience for callers that cannot hand over a workspace, and it
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocator of any kind).
+ *   Arguments, layouts and outputs as moe_route.  Limits: 1 <= T <=
+ *   MOE_ROUTE_STATIC_MAX_T, 1 <= E <= 512, 1 <= top_k <= min(E, 32); a T
+ *   above the limit returns MOE_ERR_STATIC before any CUDA call.  T = 0 is a
+ *   no-op returning MOE_OK.  The rechecked-candidate counter in the scratch
+ *   is cleared on the stream at every call; everything else is overwritten.
+ *   Concurrency: every call on a device shares the one scratch array, so two
+ *   calls whose kernels overlap on the GPU (different streams, or different
+ *   host threads without ordering) race and may return wrong routes.  Order
+ *   them on one stream.
+ */
+#define MOE_ROUTE_STATIC_MAX_T 8
+#define MOE_ROUTE_STATIC_BYTES (128 * 1024)
+int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias,
+                     int E, int top_k, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                     int32_t* perm, void* stream);
 
 /*
  * Full layer for a decode window, 1 <= T <= MOE_DECODE_MAX_T: router, grouping,

@@ -38,11 +38,13 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_RANGE = 0, -1, -2, -3
 MOE_ERR_WS, MOE_ERR_CUDA, MOE_ERR_SLOT, MOE_ERR_TIMEOUT = -4, -5, -6, -7
+MOE_ERR_STATIC = -8
 MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T = 8, 8192
+MOE_ROUTE_STATIC_MAX_T, MOE_ROUTE_STATIC_BYTES = 8, 128 * 1024
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",
            "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
-           "moe_set_stage_events", "moe_launch_count", "moe_timeout_site")
+           "moe_set_stage_events", "moe_launch_count", "moe_timeout_site", "moe_route_static")
 
 
 class RouteOut(ctypes.Structure):
@@ -90,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.moe_launch_count.argtypes = []
         L.moe_timeout_site.restype = i32
         L.moe_timeout_site.argtypes = [P]
+        L.moe_route_static.restype = i32
+        L.moe_route_static.argtypes = [P, i32, i32, P, P, i32, i32, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -132,6 +136,17 @@ def moe_route(x, router_w, router_bias, top_k, topk_idx, topk_w, expert_offsets,
                          _ptr(topk_w), _ptr(expert_offsets), _ptr(perm), _ptr(ws), ws.numel() * ws.element_size(),
                          _stream(stream))
     return _check(rc, "moe_route", raise_on_error)
+
+
+def moe_route_static(x, router_w, router_bias, top_k, topk_idx, topk_w, expert_offsets, perm,
+                     stream=None, raise_on_error=True) -> int:
+    """moe_route with the library's fixed device scratch instead of a workspace
+    (T <= MOE_ROUTE_STATIC_MAX_T).  Calls that overlap on the GPU race."""
+    T, H = x.shape
+    E = router_w.shape[0]
+    rc = lib().moe_route_static(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, top_k, _ptr(topk_idx),
+                                _ptr(topk_w), _ptr(expert_offsets), _ptr(perm), _stream(stream))
+    return _check(rc, "moe_route_static", raise_on_error)
 
 
 def _forward(fn, name, desc, arena, slot_table, L, layer, x, router_w, router_bias, top_k, residual, out,

@@ -515,6 +515,50 @@ int moe_route(const uint16_t* x, int T, int H, const float* router_w, const floa
                         static_cast<uint8_t*>(ws), L, false, nullptr, 0, static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// Scratch of moe_route_static: one fixed array per device, no allocation.
+static __device__ __align__(256) uint8_t g_route_scratch[MOE_ROUTE_STATIC_BYTES];
+
+namespace {
+void* g_route_scratch_addr[256];  // per device, filled on first use under g_mu
+
+// Address of this device's g_route_scratch, looked up once with the device current.
+int route_scratch(uint8_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!g_route_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        if (!aligned(p, kAlign)) return MOE_ERR_CUDA;
+        g_route_scratch_addr[dev] = p;
+    }
+    *out = static_cast<uint8_t*>(g_route_scratch_addr[dev]);
+    return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias, int E,
+                     int top_k, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                     void* stream) {
+    if (T > MOE_ROUTE_STATIC_MAX_T) return MOE_ERR_STATIC;
+    int rc = check_route_args(x, T, H, router_w, E, top_k, reinterpret_cast<const void*>(kAlign),
+                              MOE_ROUTE_STATIC_MAX_T);
+    if (rc) return rc;
+    if (!topk_idx || !topk_w || !expert_offsets || !perm) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    const Ws L = ws_layout(T, E, top_k, H, 32);
+    if (L.xp > MOE_ROUTE_STATIC_BYTES) return MOE_ERR_STATIC;  // the router and grouping use [0, xp) only
+    uint8_t* scratch = nullptr;
+    rc = route_scratch(&scratch);
+    if (rc) return rc;
+    return launch_route(x, T, H, router_w, router_bias, E, top_k, topk_idx, topk_w, expert_offsets, perm, nullptr,
+                        scratch, L, false, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
 static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L,
                    int layer, const uint16_t* x, int T, const float* router_w, const float* router_bias, int E,
                    int top_k, int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
@@ -605,6 +649,7 @@ const char* moe_strerror(int code) {
         case MOE_ERR_CUDA: return "CUDA launch or query failed";
         case MOE_ERR_SLOT: return "a selected expert has no valid arena slot (it contributed zero)";
         case MOE_ERR_TIMEOUT: return "a bounded device-side wait expired";
+        case MOE_ERR_STATIC: return "size beyond the fixed scratch of moe_route_static (T > MOE_ROUTE_STATIC_MAX_T)";
         default: return "unknown error code";
     }
 }

@@ -109,3 +109,15 @@ def test_rank_experts_matches_oracle(lib):
 def test_strerror_covers_codes(lib):
     msgs = {M.strerror(c) for c in range(-7, 1)}
     assert len(msgs) == 8 and "unknown" in M.strerror(-99)
+
+
+def test_route_static_checks(lib):
+    # beyond the fixed scratch: rejected before any CUDA call, with its own code
+    assert lib.moe_route_static(FAKE, M.MOE_ROUTE_STATIC_MAX_T + 1, 2048, FAKE, None, 512, 10, FAKE, FAKE, FAKE,
+                                FAKE, None) == M.MOE_ERR_STATIC
+    assert "MOE_ROUTE_STATIC_MAX_T" in M.strerror(M.MOE_ERR_STATIC)
+    assert lib.moe_route_static(FAKE, 5, 2048, FAKE, None, 513, 10, FAKE, FAKE, FAKE, FAKE, None) == M.MOE_ERR_RANGE
+    assert lib.moe_route_static(FAKE, 5, 2048, FAKE, None, 512, 10, None, FAKE, FAKE, FAKE, None) == M.MOE_ERR_ARG
+    assert lib.moe_route_static(FAKE + 2, 5, 2048, FAKE, None, 512, 10, FAKE, FAKE, FAKE, FAKE, None) \
+        == M.MOE_ERR_ARG
+    assert lib.moe_route_static(FAKE, 0, 2048, FAKE, None, 512, 10, FAKE, FAKE, FAKE, FAKE, None) == M.MOE_OK

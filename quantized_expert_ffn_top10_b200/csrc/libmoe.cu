@@ -22,7 +22,7 @@ constexpr size_t kAlign = 256;
 inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, total;
+    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -50,6 +50,7 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.xp = put(P * H * 2);
     w.h = put(P * I * (small ? 4 : 2));  // decode keeps h and Y in fp32, prefill in bf16
     w.y = put(P * H * (small ? 4 : 2));
+    w.rec = put(small ? (size_t)DF_NREP * T * E * 16 : 0);  // fused decode: replicated (logit, bound) records
     w.total = o;
     return w;
 }
@@ -61,6 +62,7 @@ std::vector<cudaEvent_t> g_stage_ev;  // measurement hook, see moe_set_stage_eve
 std::atomic<uint64_t> g_launches{0};
 uint64_t g_init_mask[4] = {0, 0, 0, 0};  // devices whose kernel attributes are set
 int g_df_grid[256];                     // fused-decode grid (one CTA per SM) per device, 0 = unusable
+int g_df_maxdyn[256];                   // its dynamic shared-memory limit per device
 constexpr int kDfMaxH = 2560;           // largest H the fused decode kernel stages
 
 inline void stage(int i, cudaStream_t st) {
@@ -188,27 +190,30 @@ bool tmap_codes(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_b
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// codes of one matrix, 16-row boxes of 128 bytes with 128-byte swizzle (fused decode staging)
-bool tmap_codes_sw(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t n_slots,
-                   int64_t slot_bytes) {
-    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_slots};
-    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)slot_bytes};
-    cuuint32_t box[3] = {128, 16, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+// Gate and up codes of every slot as one 5-D tensor: (128-byte chunk, chunk
+// index, row, matrix, slot); a box is 16 rows x one chunk of both matrices,
+// landing as [matrix][row][128 B] with the 128-byte swizzle.
+bool tmap_codes_gu(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t mat_stride,
+                   int64_t n_slots, int64_t slot_bytes) {
+    cuuint64_t dims[5] = {128, (cuuint64_t)(row_bytes / 128), (cuuint64_t)rows, 2, (cuuint64_t)n_slots};
+    cuuint64_t strides[4] = {128, (cuuint64_t)row_bytes, (cuuint64_t)mat_stride, (cuuint64_t)slot_bytes};
+    cuuint32_t box[5] = {128, 1, 16, 2, 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<uint8_t*>(base), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp16 scales of one matrix [n_slots][rows][K/32], box (kb/32) x 16 x 1
-bool tmap_scales(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t K, int64_t n_slots, int64_t slot_bytes,
-                 int kb) {
-    cuuint64_t dims[3] = {(cuuint64_t)(K / 32), (cuuint64_t)rows, (cuuint64_t)n_slots};
-    cuuint64_t strides[2] = {(cuuint64_t)(K / 32 * 2), (cuuint64_t)slot_bytes};
-    cuuint32_t box[3] = {(cuuint32_t)(kb / 32), 16, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+// W_d codes of every slot as a 4-D tensor (128-byte chunk, chunk index, row,
+// slot); a box is 16 rows x all chunks of a row, landing as [row][chunk][128 B].
+bool tmap_codes_d(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t n_slots,
+                  int64_t slot_bytes) {
+    cuuint64_t dims[4] = {128, (cuuint64_t)(row_bytes / 128), (cuuint64_t)rows, (cuuint64_t)n_slots};
+    cuuint64_t strides[3] = {128, (cuuint64_t)row_bytes, (cuuint64_t)slot_bytes};
+    cuuint32_t box[4] = {128, (cuuint32_t)(row_bytes / 128), 16, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -235,15 +240,17 @@ int ensure_init() {
     chk(set_smem(k_prefill_gemm<0, 4, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 2, 2>, PfCfg<0>::SMEM));
     chk(set_smem(k_prefill_gemm<0, 2, 4>, PfCfg<0>::SMEM)); chk(set_smem(k_prefill_gemm<0, 4, 2>, PfCfg<0>::SMEM));
     chk(set_smem(k_prefill_gemm<1, 4, 4>, PfCfg<1>::SMEM)); chk(set_smem(k_prefill_gemm<1, 2, 2>, PfCfg<1>::SMEM));
-    const int dfs = df_smem_bytes(kDfMaxH);
-    chk(set_smem(k_decode_fused<4, 4, 4>, dfs)); chk(set_smem(k_decode_fused<2, 2, 4>, dfs));
-    chk(set_smem(k_decode_fused<4, 4, 2>, dfs)); chk(set_smem(k_decode_fused<2, 2, 2>, dfs));
-    chk(set_smem(k_decode_fused<2, 4, 4>, dfs)); chk(set_smem(k_decode_fused<4, 2, 4>, dfs));
-    chk(set_smem(k_decode_fused<2, 4, 2>, dfs)); chk(set_smem(k_decode_fused<4, 2, 2>, dfs));
+    // fused decode: all the shared memory a CTA can have, less the kernel's static arrays
+    cudaFuncAttributes fa{};
+    chk(cudaFuncGetAttributes(&fa, k_decode_fused<4, 4>));
+    const int dfs = DF_SMEM_LIMIT - (int)fa.sharedSizeBytes;
+    chk(set_smem(k_decode_fused<4, 4>, dfs)); chk(set_smem(k_decode_fused<4, 2>, dfs));
+    chk(set_smem(k_decode_fused<2, 4>, dfs)); chk(set_smem(k_decode_fused<2, 2>, dfs));
     int nsm = 0, per = 0;
     chk(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-    chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4, 4>, DF_THREADS, dfs));
+    chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4>, DF_THREADS, dfs));
     g_df_grid[dev] = (per >= 1) ? nsm : 0;
+    g_df_maxdyn[dev] = dfs;
     if (e != cudaSuccess || !encoder()) return MOE_ERR_CUDA;
     g_init_mask[dev >> 6] |= 1ull << (dev & 63);
     return MOE_OK;
@@ -318,37 +325,38 @@ void launch_down(const DecodeArgs& a, int umax, int T, cudaStream_t st) {
 // Shapes the fused decode kernel stages: gate/up K-chunks of min(H, 1024)
 // with 128-byte code rows per chunk and 16-byte scale rows; down rows of
 // 128-byte multiples; everything within one ring slot and the smem plan.
-bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k) {
+// Whether the fused decode kernel takes this window; fills its shared-memory plan.
+bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k, DfPlan* plan, int* dyn, int* epc) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || g_df_grid[dev] < 1) return false;
-    const int H = d->H, I = d->I;
-    if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH || H % DF_CHUNK || I % 256) return false;
-    if ((I * d->bits_down / 8) % 128) return false;
-    // one phase-D unit: W_d rows, scales, h and half-block sums of up to T pairs
-    const int hs = std::min(T, DF_HSTAGE);
-    if ((I * d->bits_down / 8 / 128) * 2048 + 16 * (I / 32) * 2 + hs * I * 2 + hs * (I / 16) * 4 > DF_SLOT) return false;
-    if ((DF_CHUNK * d->bits_gate / 8 / 128 + DF_CHUNK * d->bits_up / 8 / 128) * 2048 + 2 * 16 * (DF_CHUNK / 32) * 2 >
-        DF_SLOT)
-        return false;
-    return true;
+    const int H = d->H, I = d->I, G = g_df_grid[dev];
+    if (d->bits_gate != d->bits_up) return false;  // one unit shape for gate and up
+    if (d->off_codes[1] <= d->off_codes[0]) return false;  // gate and up codes as one tensor
+    if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH) return false;
+    if (H % df_ck(d->bits_gate) || H % 256 || I % 256 || I / 32 > DF_MAX_NBD) return false;
+    const int wd_row = I * d->bits_down / 8;  // bytes of a W_d row: one or two 128-byte boxes
+    if (wd_row % 128 || wd_row > DF_CODE_SLOT / 16) return false;
+    *epc = (E + G - 1) / G;
+    if (*epc > DF_MAX_EPC) return false;
+    return df_plan(*plan, T, T * k, E, H, I, d->bits_gate, *epc, G, g_df_maxdyn[dev], dyn);
 }
 
-template <int BG, int BU, int BD>
-cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int grid, cudaStream_t st) {
+template <int BGU, int BD>
+cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int grid, int dyn, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(DF_THREADS);
-    cfg.dynamicSmemBytes = df_smem_bytes(kDfMaxH);
+    cfg.dynamicSmemBytes = dyn;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeCooperative;  // all CTAs co-resident: the grid barriers rely on it
     at[0].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_fused<BG, BU, BD>, tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], a);
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<BGU, BD>, tm[0], tm[1], a);
 }
 
-int run_decode_fused(const LayerCall& c) {
+int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     const moe_arena_desc* d = c.d;
     const int H = d->H, I = d->I;
     const Ws L = ws_layout(c.T, c.E, c.k, H, I);
@@ -359,7 +367,7 @@ int run_decode_fused(const LayerCall& c) {
     a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = d->n_slots; a.slot_bytes = d->slot_bytes;
     for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
     a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.residual;
-    a.bits_g = d->bits_gate; a.bits_u = d->bits_up; a.bits_d = d->bits_down;
+    a.epc = epc;
     a.x = c.x; a.W = c.W; a.b = c.b; a.out = c.out; a.hist = c.hist;
     a.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
     a.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
@@ -367,36 +375,27 @@ int run_decode_fused(const LayerCall& c) {
     a.perm = (ro && ro->perm) ? ro->perm : reinterpret_cast<int32_t*>(c.ws + L.perm);
     a.nrechk = (ro && ro->n_rechecked) ? ro->n_rechecked : reinterpret_cast<int32_t*>(c.ws + L.nrechk);
     a.logit = reinterpret_cast<double*>(c.ws + L.logit);
-    a.absum = reinterpret_cast<double*>(c.ws + L.absum);
     a.wnorm = reinterpret_cast<float*>(c.ws + L.cmax);
     a.hB = reinterpret_cast<uint16_t*>(c.ws + L.h);
-    a.hC = reinterpret_cast<float*>(c.ws + L.y);
     a.bar = reinterpret_cast<unsigned int*>(c.ws + L.meta + 8);
-    CUtensorMap tm[6];
+    a.rec = reinterpret_cast<double2*>(c.ws + L.rec);
+    a.pl = plan;
+    CUtensorMap tm[2];
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
-    const int chunk = DF_CHUNK;
-    if (!tmap_codes_sw(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8, ns, sb) ||
-        !tmap_codes_sw(&tm[1], c.arena + d->off_codes[1], I, (int64_t)H * d->bits_up / 8, ns, sb) ||
-        !tmap_codes_sw(&tm[2], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb) ||
-        !tmap_scales(&tm[3], c.arena + d->off_scales[0], I, H, ns, sb, chunk) ||
-        !tmap_scales(&tm[4], c.arena + d->off_scales[1], I, H, ns, sb, chunk) ||
-        !tmap_scales(&tm[5], c.arena + d->off_scales[2], H, I, ns, sb, I))
+    if (!tmap_codes_gu(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8,
+                       d->off_codes[1] - d->off_codes[0], ns, sb) ||
+        !tmap_codes_d(&tm[1], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb))
         return MOE_ERR_CUDA;
-    if (cudaMemsetAsync(a.bar, 0, 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
+    if (cudaMemsetAsync(a.bar, 0, 33 * 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
         return MOE_ERR_CUDA;
     stage(0, c.st);
     const int grid = g_df_grid[dev];
-    const int key = d->bits_gate * 100 + d->bits_up * 10 + d->bits_down;
     cudaError_t e;
-    switch (key) {
-        case 444: e = launch_fused<4, 4, 4>(tm, a, grid, c.st); break;
-        case 224: e = launch_fused<2, 2, 4>(tm, a, grid, c.st); break;
-        case 442: e = launch_fused<4, 4, 2>(tm, a, grid, c.st); break;
-        case 222: e = launch_fused<2, 2, 2>(tm, a, grid, c.st); break;
-        case 244: e = launch_fused<2, 4, 4>(tm, a, grid, c.st); break;
-        case 424: e = launch_fused<4, 2, 4>(tm, a, grid, c.st); break;
-        case 242: e = launch_fused<2, 4, 2>(tm, a, grid, c.st); break;
-        default: e = launch_fused<4, 2, 2>(tm, a, grid, c.st); break;
+    switch (d->bits_gate * 10 + d->bits_down) {
+        case 44: e = launch_fused<4, 4>(tm, a, grid, dyn, c.st); break;
+        case 42: e = launch_fused<4, 2>(tm, a, grid, dyn, c.st); break;
+        case 24: e = launch_fused<2, 4>(tm, a, grid, dyn, c.st); break;
+        default: e = launch_fused<2, 2>(tm, a, grid, dyn, c.st); break;
     }
     for (int i = 1; i < 5; ++i) stage(i, c.st);  // one kernel: the stages collapse onto its end
     count(1);
@@ -404,7 +403,9 @@ int run_decode_fused(const LayerCall& c) {
 }
 
 int run_decode(const LayerCall& c) {
-    if (fused_decode_ok(c.d, c.T, c.E, c.k)) return run_decode_fused(c);
+    DfPlan plan;
+    int dyn = 0, epc = 0;
+    if (fused_decode_ok(c.d, c.T, c.E, c.k, &plan, &dyn, &epc)) return run_decode_fused(c, plan, dyn, epc);
     const moe_arena_desc* d = c.d;
     const Ws L = ws_layout(c.T, c.E, c.k, d->H, d->I);
     Routed r;

@@ -510,8 +510,9 @@ struct DfDRegs {
 
 // The unit's codes sit as [16 rows][nbox 128-byte chunks] with the TMA
 // 128-byte swizzle keyed on the 128-byte line index (row * nbox + chunk).
-template <int BD>
-__device__ __forceinline__ void df_stage_d(const uint8_t* code, const uint8_t* sc, int nblk, int nbox, DfDRegs& r) {
+template <int BD, int nblk>
+__device__ __forceinline__ void df_stage_d(const uint8_t* code, const uint8_t* sc, DfDRegs& r) {
+    constexpr int nbox = nblk * BD / 32;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, key16 = (g & 7) << 4;
     if (BD == 4) {
         // blocks j, j + 1 of rows 0-7 / 8-15: matrices (rows 0-7, j), (8-15, j), (0-7, j+1), (8-15, j+1)
@@ -533,7 +534,7 @@ __device__ __forceinline__ void df_stage_d(const uint8_t* code, const uint8_t* s
             r.c1[j] = j < nblk ? ld_codes<BD>(r0 + 1024, j, q, key16) : 0u;
         }
     }
-    const int ns = nblk / 8;  // uint4 of scales per row
+    constexpr int ns = nblk / 8;  // uint4 of scales per row
 #pragma unroll
     for (int i = 0; i < DF_MAX_NBD / 8; ++i) {
         r.s0[i] = i < ns ? *reinterpret_cast<const uint4*>(sc + (g * ns + i) * 16) : make_uint4(0u, 0u, 0u, 0u);
@@ -544,9 +545,9 @@ __device__ __forceinline__ void df_stage_d(const uint8_t* code, const uint8_t* s
 // acc (features g, g + 8; pair columns 2q, 2q + 1) = W_d rows x h of the
 // expert's n pairs.  hs: staged h of the first pair [n][hstride bytes], in
 // fragment order; hsum: per pair and block, the sum of its 32 h values.
-template <int BD>
+template <int BD, int nblk>
 __device__ __forceinline__ void df_compute_d(const DfDRegs& r, const uint8_t* hs, int hstride, const float* hsum,
-                                             int nblk, int n, float (&acc)[4]) {
+                                             int n, float (&acc)[4]) {
     constexpr float kOff = 128.f + (float)(1 << (BD - 1));
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const bool col_ok = g < n, ok0 = 2 * q < n, ok1 = 2 * q + 1 < n;
@@ -574,7 +575,7 @@ __device__ __forceinline__ void df_compute_d(const DfDRegs& r, const uint8_t* hs
 
 // ---------------------------------------------------------------- the kernel
 
-template <int BGU, int BD>
+template <int BGU, int BD, int NBD>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     k_decode_fused(const __grid_constant__ CUtensorMap tgu, const __grid_constant__ CUtensorMap tcd,
                    DecodeFusedArgs a) {
@@ -787,7 +788,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     // ---- C: gate/up + SwiGLU.  A grid barrier separates C from D, so each phase
     // is balanced on its own: every CTA takes an equal share of the 16-row
     // gate/up tiles, contiguous in (expert, row) order.
-    const int tiles_e = I / 16, NCH = H / CK, NFT = H / DF_FT, nblk_d = I / 32;
+    const int tiles_e = I / 16, NCH = H / CK, NFT = H / DF_FT;
+    constexpr int nblk_d = NBD, nbox_d = NBD * BD / 32;  // W_d row: quant blocks, 128-byte chunks
     const int nuq = alive ? *rt.n_uniq : 0;
     const int R = nuq * tiles_e;
     const int r0 = (int)((int64_t)cta * R / G), r1 = (int)((int64_t)(cta + 1) * R / G);
@@ -805,7 +807,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     const int nftc = df_nft(cta, NFT, G);
     const int ndw = (alive && nuq > warp) ? (nuq - warp + DF_WARPS - 1) / DF_WARPS : 0;
     const int S = nC + nftc * ndw;
-    const int nbox_d = I * BD / 8 / 128;
     const uint32_t bytes_c = 2u * 2048u, bytes_d = (uint32_t)(nbox_d * 2048);
     const int64_t srow_g = H / 32 * 2, srow_d = nblk_d * 2;  // bytes of a scale row (gate/up, down)
 
@@ -965,14 +966,14 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             const bool valid = rt.u_sl[ui] >= 0;
             DfDRegs dr;
             if (valid)
-                df_stage_d<BD>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT, scr + (warp * DF_NBUF + b) * pl.sc_slot,
-                               nblk_d, nbox_d, dr);
+                df_stage_d<BD, NBD>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT,
+                                    scr + (warp * DF_NBUF + b) * pl.sc_slot, dr);
             __syncwarp();
             if (issued < S) issue(issued++);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             if (valid)
-                df_compute_d<BD>(dr, hs + (size_t)pos0 * pl.hs_stride, pl.hs_stride, hsum + (size_t)pos0 * nblk_d,
-                                 nblk_d, n, acc);
+                df_compute_d<BD, NBD>(dr, hs + (size_t)pos0 * pl.hs_stride, pl.hs_stride,
+                                      hsum + (size_t)pos0 * nblk_d, n, acc);
 #pragma unroll
             for (int z = 0; z < 2; ++z) {  // y for pair columns 2q, 2q+1 (when they exist), features g, g+8
                 const int jj = 2 * q + z;

@@ -242,13 +242,14 @@ int ensure_init() {
     chk(set_smem(k_prefill_gemm<1, 4, 4>, PfCfg<1>::SMEM)); chk(set_smem(k_prefill_gemm<1, 2, 2>, PfCfg<1>::SMEM));
     // fused decode: all the shared memory a CTA can have, less the kernel's static arrays
     cudaFuncAttributes fa{};
-    chk(cudaFuncGetAttributes(&fa, k_decode_fused<4, 4>));
+    chk(cudaFuncGetAttributes(&fa, k_decode_fused<4, 4, 16>));
     const int dfs = DF_SMEM_LIMIT - (int)fa.sharedSizeBytes;
-    chk(set_smem(k_decode_fused<4, 4>, dfs)); chk(set_smem(k_decode_fused<4, 2>, dfs));
-    chk(set_smem(k_decode_fused<2, 4>, dfs)); chk(set_smem(k_decode_fused<2, 2>, dfs));
+    chk(set_smem(k_decode_fused<4, 4, 16>, dfs)); chk(set_smem(k_decode_fused<4, 4, 8>, dfs));
+    chk(set_smem(k_decode_fused<4, 2, 16>, dfs)); chk(set_smem(k_decode_fused<2, 4, 16>, dfs));
+    chk(set_smem(k_decode_fused<2, 4, 8>, dfs)); chk(set_smem(k_decode_fused<2, 2, 16>, dfs));
     int nsm = 0, per = 0;
     chk(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-    chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4>, DF_THREADS, dfs));
+    chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4, 16>, DF_THREADS, dfs));
     g_df_grid[dev] = (per >= 1) ? nsm : 0;
     g_df_maxdyn[dev] = dfs;
     if (e != cudaSuccess || !encoder()) return MOE_ERR_CUDA;
@@ -341,7 +342,7 @@ bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k, DfPlan* plan,
     return df_plan(*plan, T, T * k, E, H, I, d->bits_gate, *epc, G, g_df_maxdyn[dev], dyn);
 }
 
-template <int BGU, int BD>
+template <int BGU, int BD, int NBD>
 cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int grid, int dyn, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
@@ -353,7 +354,7 @@ cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int gr
     at[0].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_fused<BGU, BD>, tm[0], tm[1], a);
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<BGU, BD, NBD>, tm[0], tm[1], a);
 }
 
 int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
@@ -391,11 +392,13 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     stage(0, c.st);
     const int grid = g_df_grid[dev];
     cudaError_t e;
-    switch (d->bits_gate * 10 + d->bits_down) {
-        case 44: e = launch_fused<4, 4>(tm, a, grid, dyn, c.st); break;
-        case 42: e = launch_fused<4, 2>(tm, a, grid, dyn, c.st); break;
-        case 24: e = launch_fused<2, 4>(tm, a, grid, dyn, c.st); break;
-        default: e = launch_fused<2, 2>(tm, a, grid, dyn, c.st); break;
+    switch (d->bits_gate * 1000 + d->bits_down * 100 + I / 32) {  // I / 32 blocks per W_d row
+        case 4416: e = launch_fused<4, 4, 16>(tm, a, grid, dyn, c.st); break;
+        case 4408: e = launch_fused<4, 4, 8>(tm, a, grid, dyn, c.st); break;
+        case 4216: e = launch_fused<4, 2, 16>(tm, a, grid, dyn, c.st); break;
+        case 2416: e = launch_fused<2, 4, 16>(tm, a, grid, dyn, c.st); break;
+        case 2408: e = launch_fused<2, 4, 8>(tm, a, grid, dyn, c.st); break;
+        default: e = launch_fused<2, 2, 16>(tm, a, grid, dyn, c.st); break;
     }
     for (int i = 1; i < 5; ++i) stage(i, c.st);  // one kernel: the stages collapse onto its end
     count(1);

@@ -50,6 +50,24 @@ def parse():
     return p.parse_args()
 
 
+def profiled_traffic(summary: str, sources) -> int | None:
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or None
+    when the kernel's sources changed since that capture."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(root, "profiles", summary)).read()
+        m = hashlib.sha256()
+        for f in sources:
+            m.update(open(os.path.join(root, "quantized_expert_ffn_top10_b200", "csrc", f), "rb").read())
+        fields = dict(l.split(": ", 1) for l in text.splitlines() if l.startswith(("traffic_", "kernel_sources")))
+        if fields.get("kernel_sources_sha256", "").strip() != m.hexdigest():
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -117,7 +135,7 @@ class Layers:
         import torch
         import moe_synth as S
         import quantized_expert_ffn_top10_b200 as M
-        self.cfg = S.config(cfg.name, L=NL, seed=cfg.seed + 1000 * rank)
+        self.cfg = S.config(cfg.name, L=NL, seed=replica_seed(cfg.seed, rank))
         c = self.cfg
         self.NL = NL
         self.desc = c.desc()
@@ -182,9 +200,7 @@ def time_graphs(layers: Layers, steps: int, warmup: int, dev: int, dist):
     ms = e0.elapsed_time(e1)
     if dist:
         dist.barrier()
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ms)
     # stage durations of each graph's last replay (all inside the timed region when steps >= NL)
     try:
         stages = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]
@@ -223,11 +239,7 @@ def time_e2e(layers: Layers, steps: int, warmup: int, dist):
         step(warmup + i)
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, e0.elapsed_time(e1))
     nbytes = xh[0].numel() * 2
     return ms, nbytes, nbytes
 
@@ -275,6 +287,29 @@ def cores():
 def rank_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def max_over_ranks(dist, ms: float) -> float:
+    """The slowest rank's time (every rank gets it); the value itself when
+    running alone.  NCCL reduces a device tensor, gloo a host one."""
+    if not dist:
+        return ms
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Units of all ranks per second, timed by the slowest rank (weak scaling:
+    every rank processes the same amount of independent work)."""
+    return units_per_rank * world / (ms / 1e3)
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank's replica draws its own inputs and weights."""
+    return base_seed + 1000 * rank
 
 
 def decode_bytes(c, distinct: int):
@@ -334,8 +369,7 @@ def decode_section(args, rank, local, world, dist, hbm, src, K, W):
     dl = Layers(S.config("decode"), NLd, rank)
     c = dl.cfg
     ms, stages, distinct, per_call, clk = time_graphs(dl, K, W, local, dist)
-    tok = c.T * K * world
-    value = tok / (ms / 1e3)
+    value = whole_job_rate(c.T * K, world, ms)
     fused = per_call == 1  # the decode layer is one kernel: its roofline is the layer's
     gu_ms = statistics.mean(s[0] + s[1] + s[2] + s[3] for s in stages) if fused else statistics.mean(s[1] for s in stages)
     gu_bytes = statistics.mean((decode_bytes if fused else gateup_bytes)(c, d) for d in distinct)
@@ -352,14 +386,17 @@ def decode_section(args, rank, local, world, dist, hbm, src, K, W):
         "roofline": {"bound": "hbm", "kernel": "k_decode_fused (whole layer)" if fused else "decode gate/up + SwiGLU",
                      "achieved": round(gu_bytes / (gu_ms * 1e6), 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(gu_bytes / (gu_ms * 1e6) / hbm, 4),
-                     "traffic": None, "peak_source": src, "ms": round(gu_ms, 5),
+                     "traffic": profiled_traffic("k_decode_fused_decode_T5.md",
+                                                 ("common.cuh", "perm.cuh", "router.cuh", "decode_fused.cuh"))
+                     if fused else None,
+                     "peak_source": src, "ms": round(gu_ms, 5),
                      "bytes": int(gu_bytes)},
         "layer_roofline": {"bound": "hbm", "achieved": round(layer_bytes / (ms / K * 1e6), 1), "peak": hbm,
                            "unit": "GB/s", "frac": round(layer_bytes / (ms / K * 1e6) / hbm, 4),
                            "frac_of_8tbs": round(layer_bytes / (ms / K * 1e6) / 8000.0, 4),
                            "bytes_per_layer": int(layer_bytes), "distinct_experts": statistics.mean(distinct),
                            "stage_ms": [round(statistics.mean(s[j] for s in stages), 5) for j in range(4)]},
-        "e2e": {"value": round(c.T * K * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_rate(c.T * K, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": per_call * K,
         "clocks": clk,
@@ -385,19 +422,21 @@ def prefill_section(args, line, rank, local, world, dist, tc_burst, tc_sus, src,
         flops = f1 + f2 + 2.0 * cp.T * cp.E * cp.H
         e2p, h2p, d2p = time_e2e(pl, max(2, Kp // 4), 2, dist)
         line["prefill"] = {
-            "value": round(cp.T * Kp * world / (msp / 1e3), 1), "unit": "tokens/s", "steps": Kp,
+            "value": round(whole_job_rate(cp.T * Kp, world, msp), 1), "unit": "tokens/s", "steps": Kp,
             "ms_per_step": round(msp / Kp, 4),
             "workload": "prefill chunk: 1 layer, E=512, top_k=10, H=2048, I=512, T=8192, 4-bit, Gaussian router",
             "roofline": {"bound": "tensor", "kernel": "prefill gate/up grouped GEMM + SwiGLU",
                          "achieved": round(f1 / (g1 * 1e9), 1), "peak": tc_sus, "unit": "TFLOP/s",
-                         "frac": round(f1 / (g1 * 1e9) / tc_sus, 4), "traffic": None, "peak_source": src + " sustained",
+                         "frac": round(f1 / (g1 * 1e9) / tc_sus, 4),
+                         "traffic": profiled_traffic("k_prefill_gemm_prefill_T8192.md", ("common.cuh", "prefill.cuh")),
+                         "peak_source": src + " sustained",
                          "ms": round(g1, 4)},
             "gemm2": {"achieved": round(f2 / (g2 * 1e9), 1), "unit": "TFLOP/s", "frac": round(f2 / (g2 * 1e9) / tc_sus, 4),
                       "ms": round(g2, 4)},
             "layer_tc_frac": round(flops / (msp / Kp * 1e9) / tc_sus, 4),
             "layer_tc_frac_burst": round(flops / (msp / Kp * 1e9) / tc_burst, 4),
             "stage_ms": [round(statistics.mean(s[j] for s in stp), 4) for j in range(4)],
-            "e2e": {"value": round(cp.T * max(2, Kp // 4) * world / (e2p / 1e3), 1), "unit": "tokens/s",
+            "e2e": {"value": round(whole_job_rate(cp.T * max(2, Kp // 4), world, e2p), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2p, "d2h_bytes_per_step": d2p},
             "gpu_launches": pcp * Kp, "clocks": clkp,
         }

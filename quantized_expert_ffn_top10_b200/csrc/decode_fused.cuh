@@ -48,6 +48,7 @@
 #define DF_MAX_EPC 8       // router experts per CTA (rows of the fp64 MMA)
 #define DF_MAX_NBD 16      // quant blocks of a W_d row (I <= 512 at 4 bits)
 #define DF_SMEM_LIMIT (227 * 1024)
+#define DF_BAR_WORDS (32 * 18)  // grid barrier: 16 group counters, the top counter, the flag
 #define DF_NREP 8          // copies of the (logit, bound) records that phase B reads
 
 // Shared-memory layout, computed on the host (df_plan) and passed in; offsets
@@ -57,7 +58,7 @@ struct DfPlan {
     int r1_off;                 // C: xb, xc, partials | D: h, hsum, ypair
     int xc_off, part_off, n_part, part_bytes;
     int hs_stride, hsum_off, ypair_off;
-    int route_off, bar_off, total;
+    int route_off, stab_off, bar_off, total;
     // phase A (code ring, free then): x rows, W_r rows, per-warp sums, x block sums
     int a_ws_off, a_sp_off, a_w2_off, a_xp_off;
     // phase B (code ring): per-token scratch, expert counts and offsets
@@ -86,7 +87,7 @@ struct DecodeFusedArgs {
     float* wnorm;            // [E] upper bounds of ||W[e]||_2 (workspace)
     double2* rec;            // [DF_NREP][T][E] (logit, error bound): CTA c reads copy c % DF_NREP
     uint16_t* hB;            // [P][I] bf16, MMA-fragment order within each 32-block
-    unsigned int* bar;       // grid barrier: [0] arrivals, [32] completed phase (zeroed before launch)
+    unsigned int* bar;       // grid barrier counters and flag, DF_BAR_WORDS words (zeroed before launch)
     DfPlan pl;
 };
 
@@ -130,8 +131,10 @@ __host__ inline bool df_plan(DfPlan& p, int T, int P, int E, int H, int I, int b
     o = df_al(std::max(c_end, d_end), 16);
     p.route_off = o;
     o += df_al((8 * P + 4) * 4, 16);
+    p.stab_off = o;  // this layer's row of the slot table
+    o += MOE_MAX_E * 4;
     p.bar_off = o;
-    o += (DF_WARPS * DF_NBUF + 1) * 8;
+    o += (DF_WARPS * DF_NBUF + 2) * 8;
     p.total = df_al(o, 128);
     // phase A inside the code ring: x rows [T][2H + 16], W_r rows [epc][4H + 16], sums
     p.a_ws_off = df_al(T * (2 * H + 16), 128);
@@ -155,24 +158,29 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
-// Grid-wide barrier over gridDim.x co-resident CTAs, phase `ph` (1, 2, ...).
-// ctr[0] counts arrivals (it only grows); the CTA that completes a phase
-// stores the phase number to ctr[32], a separate 128-byte line that the
-// others poll, so the polling does not contend with the arrivals.  Bounded:
-// on expiry the status word gets MOE_ERR_TIMEOUT and every thread of the CTA
-// sees false.
-__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned ph, int site) {
+// Grid-wide barrier over gridDim.x co-resident CTAs, phase `ph` (1, 2, ...),
+// in two levels so that no counter sees more than ~16 arrivals: CTA c arrives
+// on group counter c % DF_BAR_GROUPS; the last arrival of a group arrives on
+// the top counter; the last arrival there stores the phase to the release
+// flag, which the others poll.  Counters and flag sit on separate 128-byte
+// lines of `bar` (zeroed before launch) and only grow.  Bounded: on expiry the
+// status word gets MOE_ERR_TIMEOUT and every thread of the CTA sees false.
+#define DF_BAR_GROUPS 16
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned ph, int site) {
     __syncthreads();
     int ok = 1;
     if (threadIdx.x == 0) {
+        const unsigned G = gridDim.x, NG = min(G, (unsigned)DF_BAR_GROUPS), grp = blockIdx.x % NG;
+        const unsigned members = (G - grp + NG - 1) / NG;
+        unsigned* flag = bar + 32 * (DF_BAR_GROUPS + 1);
         __threadfence();
-        const unsigned target = ph * gridDim.x;
-        if (atomicAdd(ctr, 1u) + 1u == target) {
-            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ctr + 32), "r"(ph) : "memory");
+        if (atomicAdd(bar + 32 * grp, 1u) + 1u == ph * members &&
+            atomicAdd(bar + 32 * DF_BAR_GROUPS, 1u) + 1u == ph * NG) {
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(ph) : "memory");
         } else {
             unsigned it = 0;
-            while (ld_acquire_u32(ctr + 32) < ph) {
-                if (++it > MOE_SPIN_LIMIT) { moe_note_timeout(site, (int)(ld_acquire_u32(ctr) % 1000)); ok = 0; break; }
+            while (ld_acquire_u32(flag) < ph) {
+                if (++it > MOE_SPIN_LIMIT) { moe_note_timeout(site, (int)(ld_acquire_u32(flag) % 1000)); ok = 0; break; }
                 if (it > 16) __nanosleep(32);
             }
         }
@@ -339,7 +347,7 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
 #pragma unroll
     for (int i = 0; i < NV; ++i) m = fmax(m, v[i]);
     int r = 0;  // rank of this lane's maximum (descending, ties by lane)
-#pragma unroll
+#pragma unroll 4
     for (int j = 0; j < 32; ++j) {
         const double o = __shfl_sync(0xffffffffu, m, j);
         r += (o > m || (o == m && j < lane)) ? 1 : 0;
@@ -380,7 +388,7 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
         }
         // position of this candidate in (value desc, expert asc) order
         int rank = 0;
-#pragma unroll
+#pragma unroll 4
         for (int j = 0; j < 32; ++j) {
             const double oj = __shfl_sync(0xffffffffu, cval, j);
             const int ej = __shfl_sync(0xffffffffu, ce, j);
@@ -573,6 +581,55 @@ __device__ __forceinline__ void df_compute_d(const DfDRegs& r, const uint8_t* hs
     }
 }
 
+// The same product computed straight from the slot in a rolled loop (two
+// blocks per step): a W_d unit is used once per launch, so its code stays
+// small instead of being unrolled over all blocks.
+template <int BD, int nblk>
+__device__ __forceinline__ void df_compute_d_smem(const uint8_t* code, const uint8_t* sc, const uint8_t* hs, int hstride,
+                                                  const float* hsum, int n, float (&acc)[4]) {
+    constexpr int nbox = nblk * BD / 32;
+    constexpr float kOff = 128.f + (float)(1 << (BD - 1));
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, key16 = (g & 7) << 4;
+    const bool col_ok = g < n, ok0 = 2 * q < n, ok1 = 2 * q + 1 < n;
+    const int mrow = ((lane >> 3) & 1) * 8 + (lane & 7), jo = lane >> 4;  // ldmatrix row address of this lane
+    const uint8_t* hrow = hs + g * hstride + q * 16;
+#pragma unroll 1
+    for (int j = 0; j < nblk; j += 2) {
+        uint32_t c[2][2];  // [block j, j + 1][row g, g + 8]
+        if (BD == 4) {
+            const int jj = j + jo, line = mrow * nbox + (jj >> 3);
+            ldsm_x4(code + line * 128 + (((jj & 7) ^ (line & 7)) << 4), c[0][0], c[0][1], c[1][0], c[1][1]);
+        } else {
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                c[z][0] = ld_codes<BD>(code + g * 128, j + z, q, key16);
+                c[z][1] = ld_codes<BD>(code + g * 128 + 1024, j + z, q, key16);
+            }
+        }
+        const uint32_t sw0 = *reinterpret_cast<const uint32_t*>(sc + (g * nblk + j) * 2);  // rows g, g + 8
+        const uint32_t sw1 = *reinterpret_cast<const uint32_t*>(sc + ((g + 8) * nblk + j) * 2);
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int jb = j + z;
+            uint4 bx = make_uint4(0u, 0u, 0u, 0u);
+            if (col_ok) bx = *reinterpret_cast<const uint4*>(hrow + jb * 64);
+            const float h0 = ok0 ? hsum[(2 * q) * nblk + jb] : 0.f;
+            const float h1 = ok1 ? hsum[(2 * q + 1) * nblk + jb] : 0.f;
+            uint32_t p0[4], p1[4];
+            unpack8<BD>(c[z][0], p0);
+            unpack8<BD>(c[z][1], p1);
+            float d[4] = {-kOff * h0, -kOff * h1, -kOff * h0, -kOff * h1};
+            mma_bf16_16816(d, p0[0], p1[0], p0[1], p1[1], bx.x, bx.y);
+            mma_bf16_16816(d, p0[2], p1[2], p0[3], p1[3], bx.z, bx.w);
+            const float s0 = z ? half_hi(sw0) : half_lo(sw0), s1 = z ? half_hi(sw1) : half_lo(sw1);
+            acc[0] = fmaf(s0, d[0], acc[0]);
+            acc[1] = fmaf(s0, d[1], acc[1]);
+            acc[2] = fmaf(s1, d[2], acc[2]);
+            acc[3] = fmaf(s1, d[3], acc[3]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- the kernel
 
 template <int BGU, int BD, int NBD>
@@ -602,7 +659,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     rt.u_sl = rt.u_n + P;
     rt.n_uniq = rt.u_sl + P;
     uint64_t* full = reinterpret_cast<uint64_t*>(base + pl.bar_off);  // [DF_WARPS][DF_NBUF]
-    uint64_t* abar = full + DF_WARPS * DF_NBUF;
+    uint64_t* abar = full + DF_WARPS * DF_NBUF;  // x rows and the slot-table row
+    uint64_t* wbar = abar + 1;                   // this CTA's W_r rows
+    const int32_t* stab = reinterpret_cast<const int32_t*>(base + pl.stab_off);
     __shared__ int s_warp[33];
     __shared__ float s_xnorm[DF_TN];
     __shared__ float s_wn[DF_MAX_EPC];
@@ -613,6 +672,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < DF_WARPS * DF_NBUF; ++i) mbar_init(&full[i], 1);
         mbar_init(abar, 1);
+        mbar_init(wbar, 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -627,11 +687,14 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     uint8_t* xs = ring;
     uint8_t* ws = ring + pl.a_ws_off;
     if (tid == 0) {
-        mbar_arrive_expect_tx(abar, (uint32_t)(T * 2 * H + ne * 4 * H));
+        // the arrival completes the phase at once when ne == 0 (no bytes expected)
+        mbar_arrive_expect_tx(wbar, (uint32_t)(ne * 4 * H));
+        for (int e = 0; e < ne; ++e) bulk_load(ws + e * wstride, a.W + (size_t)(e0 + e) * H, (uint32_t)(4 * H), wbar);
+        mbar_arrive_expect_tx(abar, (uint32_t)(T * 2 * H + E * 4));
         for (int t = 0; t < T; ++t) bulk_load(xs + t * xstride, a.x + (size_t)t * H, (uint32_t)(2 * H), abar);
-        for (int e = 0; e < ne; ++e) bulk_load(ws + e * wstride, a.W + (size_t)(e0 + e) * H, (uint32_t)(4 * H), abar);
+        bulk_load(base + pl.stab_off, a.slot_table + (size_t)a.layer * E, (uint32_t)(E * 4), abar);
     }
-    bool alive = mbar_wait(abar, 0, 1, 0);
+    bool alive = mbar_wait(abar, 0, 1, 0);  // the x fragments are built while W_r is still arriving
     // x as MMA B fragments [H/32][4][T], its block sums and squares
     float* xp = reinterpret_cast<float*>(ring + pl.a_xp_off);  // [2][H/32][4][T]
     const int nxf = NB * 4 * T;
@@ -650,6 +713,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         for (int z = 0; z < 8; ++z) sq = fmaf(v[z], v[z], sq);
         xp[nxf + u] = sq;
     }
+    alive = mbar_wait(wbar, 0, 1, 1) && alive;
     if (ne > 0) {
         const int g = lane >> 2, q = lane & 3;
         const int kw = H / DF_WARPS, kb = warp * kw;
@@ -753,7 +817,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         int upos;
         const int nu = block_excl_scan((tid < E && c > 0) ? 1 : 0, &upos, s_warp);
         if (tid < E && c > 0) {
-            const int64_t sl = a.slot_table[(int64_t)a.layer * E + tid];
+            const int64_t sl = stab[tid];
             rt.u_e[upos] = tid;
             rt.u_pos[upos] = off;
             rt.u_n[upos] = c;
@@ -963,17 +1027,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             if (!mbar_wait(&full[warp * DF_NBUF + b], (uint32_t)(s / DF_NBUF) & 1u, 6, s)) { wok = false; break; }
             const int d = s - nC, rr = d / ndw, ui = warp + DF_WARPS * (d % ndw);
             const int pos0 = rt.u_pos[ui], n = rt.u_n[ui];
-            const bool valid = rt.u_sl[ui] >= 0;
-            DfDRegs dr;
-            if (valid)
-                df_stage_d<BD, NBD>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT,
-                                    scr + (warp * DF_NBUF + b) * pl.sc_slot, dr);
-            __syncwarp();
-            if (issued < S) issue(issued++);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (valid)
-                df_compute_d<BD, NBD>(dr, hs + (size_t)pos0 * pl.hs_stride, pl.hs_stride,
-                                      hsum + (size_t)pos0 * nblk_d, n, acc);
+            if (rt.u_sl[ui] >= 0)
+                df_compute_d_smem<BD, NBD>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT,
+                                           scr + (warp * DF_NBUF + b) * pl.sc_slot, hs + (size_t)pos0 * pl.hs_stride,
+                                           pl.hs_stride, hsum + (size_t)pos0 * nblk_d, n, acc);
+            __syncwarp();  // the slot's reads are done: it may be refilled
+            if (issued < S) issue(issued++);
 #pragma unroll
             for (int z = 0; z < 2; ++z) {  // y for pair columns 2q, 2q+1 (when they exist), features g, g+8
                 const int jj = 2 * q + z;

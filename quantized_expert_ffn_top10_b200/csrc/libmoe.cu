@@ -22,7 +22,7 @@ constexpr size_t kAlign = 256;
 inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, total;
+    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -51,6 +51,7 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.h = put(P * I * (small ? 4 : 2));  // decode keeps h and Y in fp32, prefill in bf16
     w.y = put(P * H * (small ? 4 : 2));
     w.rec = put(small ? (size_t)DF_NREP * T * E * 16 : 0);  // fused decode: replicated (logit, bound) records
+    w.gbar = put(small ? DF_BAR_WORDS * 4 : 0);              // fused decode: grid barrier
     w.total = o;
     return w;
 }
@@ -337,6 +338,7 @@ bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k, DfPlan* plan,
     if (H % df_ck(d->bits_gate) || H % 256 || I % 256 || I / 32 > DF_MAX_NBD) return false;
     const int wd_row = I * d->bits_down / 8;  // bytes of a W_d row: one or two 128-byte boxes
     if (wd_row % 128 || wd_row > DF_CODE_SLOT / 16) return false;
+    if (E % 4) return false;  // the slot-table row arrives by one bulk copy (16-byte multiple)
     *epc = (E + G - 1) / G;
     if (*epc > DF_MAX_EPC) return false;
     return df_plan(*plan, T, T * k, E, H, I, d->bits_gate, *epc, G, g_df_maxdyn[dev], dyn);
@@ -378,7 +380,7 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     a.logit = reinterpret_cast<double*>(c.ws + L.logit);
     a.wnorm = reinterpret_cast<float*>(c.ws + L.cmax);
     a.hB = reinterpret_cast<uint16_t*>(c.ws + L.h);
-    a.bar = reinterpret_cast<unsigned int*>(c.ws + L.meta + 8);
+    a.bar = reinterpret_cast<unsigned int*>(c.ws + L.gbar);
     a.rec = reinterpret_cast<double2*>(c.ws + L.rec);
     a.pl = plan;
     CUtensorMap tm[2];
@@ -387,7 +389,7 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
                        d->off_codes[1] - d->off_codes[0], ns, sb) ||
         !tmap_codes_d(&tm[1], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb))
         return MOE_ERR_CUDA;
-    if (cudaMemsetAsync(a.bar, 0, 33 * 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
+    if (cudaMemsetAsync(a.bar, 0, DF_BAR_WORDS * 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
         return MOE_ERR_CUDA;
     stage(0, c.st);
     const int grid = g_df_grid[dev];
@@ -408,7 +410,8 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
 int run_decode(const LayerCall& c) {
     DfPlan plan;
     int dyn = 0, epc = 0;
-    if (fused_decode_ok(c.d, c.T, c.E, c.k, &plan, &dyn, &epc)) return run_decode_fused(c, plan, dyn, epc);
+    if (aligned(c.slot_table, 16) && fused_decode_ok(c.d, c.T, c.E, c.k, &plan, &dyn, &epc))
+        return run_decode_fused(c, plan, dyn, epc);
     const moe_arena_desc* d = c.d;
     const Ws L = ws_layout(c.T, c.E, c.k, d->H, d->I);
     Routed r;

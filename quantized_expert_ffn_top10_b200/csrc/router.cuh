@@ -322,39 +322,90 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             taken |= 1u << i;
         }
     }
-    // 1) M candidates, picked by the 32-bit keys with warp reductions; a
-    //    candidate set that misses a member of the true top k only fails the
-    //    certification below.
+    // 1) Candidates by the 32-bit keys; a candidate set that misses a member of
+    //    the true top k only fails the certification below.  First try every
+    //    entry at or above theta, the M-th largest of the 32 lane maxima: at
+    //    least M entries (those maxima) reach theta, so this set holds the M
+    //    largest.  With more than 32 of them, pick exactly M by M rounds of
+    //    warp-wide argmax.
     const int M = min(min(E, k + MOE_CAND_EXTRA), 32);
     int ce = -1;
     double cval = -INFINITY, cbnd = 0.0;
-    uint32_t lkey = 0;
-    int li = -1;
-    auto rescan = [&]() {  // this lane's best untaken entry (lowest index on equal keys)
-        lkey = 0;
-        li = -1;
+    int MC = M;  // candidates held one per lane
+    bool picked = false;  // warp-uniform: the threshold set was taken
+    {
+        uint32_t lmax = 0;  // invalid entries are marked taken and have key 0
 #pragma unroll
         for (int i = 0; i < NV; ++i)
-            if (!((taken >> i) & 1u) && (li < 0 || key[i] > lkey)) { lkey = key[i]; li = i; }
-    };
-    rescan();
-    for (int j = 0; j < M; ++j) {
-        const uint32_t mk = __reduce_max_sync(0xffffffffu, lkey);
-        const uint32_t me =
-            __reduce_min_sync(0xffffffffu, (li >= 0 && lkey == mk) ? (uint32_t)(lane + 32 * li) : 0xffffffffu);
-        const int owner = (int)(me & 31u);
-        double lv = 0.0, ld = 0.0;
-        if (lane == owner) {
+            if (!((taken >> i) & 1u)) lmax = max(lmax, key[i]);
+        int r = 0;
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t o = __shfl_sync(0xffffffffu, lmax, j);
+            r += (o > lmax || (o == lmax && j < lane)) ? 1 : 0;
+        }
+        const uint32_t thk = __shfl_sync(0xffffffffu, lmax, __ffs(__ballot_sync(0xffffffffu, r == M - 1)) - 1);
+        unsigned bm[NV];
+        int nc = 0;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            bm[i] = __ballot_sync(0xffffffffu, !((taken >> i) & 1u) && key[i] >= thk);
+            nc += __popc(bm[i]);
+        }
+        if (nc <= 32) {
+            int base = 0;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                if ((bm[i] >> lane) & 1u) {
+                    const int pos = base + __popc(bm[i] & ((1u << lane) - 1));
+                    cs[pos] = lane + 32 * i;
+                    cvs[pos] = v[i];
+                    cvs[32 + pos] = dl[i];
+                }
+                base += __popc(bm[i]);
+            }
+            __syncwarp();
+            if (lane < nc) {
+                ce = cs[lane];
+                cval = cvs[lane];
+                cbnd = cvs[32 + lane];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < NV; ++i) taken |= ((bm[i] >> lane) & 1u) << i;
+            MC = nc;
+            picked = true;
+        }
+    }
+    if (!picked) {  // the threshold set was too large: M rounds of argmax
+        uint32_t lkey = 0;
+        int li = -1;
+        auto rescan = [&]() {  // this lane's best untaken entry (lowest index on equal keys)
+            lkey = 0;
+            li = -1;
 #pragma unroll
             for (int i = 0; i < NV; ++i)
-                if (i == li) { lv = v[i]; ld = dl[i]; }
-        }
-        const double bv = __shfl_sync(0xffffffffu, lv, owner);
-        const double bd = __shfl_sync(0xffffffffu, ld, owner);
-        if (lane == j) { ce = (int)me; cval = bv; cbnd = bd; }
-        if (lane == owner) {
-            taken |= 1u << li;
-            rescan();
+                if (!((taken >> i) & 1u) && (li < 0 || key[i] > lkey)) { lkey = key[i]; li = i; }
+        };
+        rescan();
+        for (int j = 0; j < M; ++j) {
+            const uint32_t mk = __reduce_max_sync(0xffffffffu, lkey);
+            const uint32_t me =
+                __reduce_min_sync(0xffffffffu, (li >= 0 && lkey == mk) ? (uint32_t)(lane + 32 * li) : 0xffffffffu);
+            const int owner = (int)(me & 31u);
+            double lv = 0.0, ld = 0.0;
+            if (lane == owner) {
+#pragma unroll
+                for (int i = 0; i < NV; ++i)
+                    if (i == li) { lv = v[i]; ld = dl[i]; }
+            }
+            const double bv = __shfl_sync(0xffffffffu, lv, owner);
+            const double bd = __shfl_sync(0xffffffffu, ld, owner);
+            if (lane == j) { ce = (int)me; cval = bv; cbnd = bd; }
+            if (lane == owner) {
+                taken |= 1u << li;
+                rescan();
+            }
         }
     }
     double rest = -INFINITY;
@@ -364,13 +415,13 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     rest = warp_max_d(rest);
 
     // 2) certified on the fast values?
-    if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
+    if (sort_and_certify(cval, cbnd, ce, MC, k, rest)) {
         write_topk(k, cval, ce, idx_out, w_out);
         return;
     }
     // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
     if (MODE == 0) {
-        for (int base = 0; base < M; base += 16) {
+        for (int base = 0; base < MC; base += 16) {
             int ej[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) ej[j] = __shfl_sync(0xffffffffu, ce, min(base + j, 31));
@@ -382,7 +433,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
                 const double xd = bf16_bits_to_f32(xr[h]);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (base + j < M) {
+                    if (base + j < MC) {
                         const double p = xd * (double)__ldg(a.W + (size_t)ej[j] * H + h);
                         acc[j] += p;
                         ab[j] += fabs(p);
@@ -390,7 +441,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                if (base + j < M) {
+                if (base + j < MC) {
                     const double s = warp_sum_d(acc[j]), sa = warp_sum_d(ab[j]);
                     const double bb = a.b ? (double)a.b[ej[j]] : 0.0;
                     if (lane == base + j) {
@@ -400,7 +451,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
                 }
             }
         }
-        if (sort_and_certify(cval, cbnd, ce, M, k, rest)) {
+        if (sort_and_certify(cval, cbnd, ce, MC, k, rest)) {
             write_topk(k, cval, ce, idx_out, w_out);
             return;
         }

@@ -15,6 +15,7 @@
 #include "perm.cuh"
 #include "prefill.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 namespace {
 
@@ -22,7 +23,8 @@ constexpr size_t kAlign = 256;
 inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, total;
+    size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, wsplit,
+        xn, slow, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -52,6 +54,9 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.y = put(P * H * (small ? 4 : 2));
     w.rec = put(small ? (size_t)DF_NREP * T * E * 16 : 0);  // fused decode: replicated (logit, bound) records
     w.gbar = put(small ? DF_BAR_WORDS * 4 : 0);              // fused decode: grid barrier
+    w.wsplit = put(small ? 0 : (size_t)3 * E * H * 2);        // chunk router: W_r as three bf16 planes
+    w.xn = put(small ? 0 : (size_t)T * 4);                     // chunk router: ||x_t|| per token
+    w.slow = put(small ? 0 : (size_t)(T + 4) * 4);             // chunk top-k: [count, tokens...] left to the slow pass
     w.total = o;
     return w;
 }
@@ -108,6 +113,9 @@ inline double gamma_n(int n, double u) { return (double)n * u / (1.0 - (double)n
 
 inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+bool tmap_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows);
+bool g_router_tc_ok[256];  // the tensor-core router kernel may run on this device (set by ensure_init)
+
 // Router + grouping on the caller's stream.  idx/w/offsets/perm may be the
 // caller's buffers or workspace.
 int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b, int E, int k, int32_t* idx,
@@ -130,11 +138,33 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
     } else {
         float* wnorm = reinterpret_cast<float*>(ws + L.cmax);
         float* logit = reinterpret_cast<float*>(ws + L.logit);
-        k_router_norms<<<(E + 7) / 8, 256, 0, st>>>(W, E, H, wnorm);
-        k_router_gemm<<<dim3((E + RG_BN - 1) / RG_BN, (T + RG_BM - 1) / RG_BM), 256, 0, st>>>(x, T, H, W, b, E, logit);
+        int dev = 0;
+        cudaGetDevice(&dev);
+        CUtensorMap tmA, tmB;
+        uint16_t* planes = reinterpret_cast<uint16_t*>(ws + L.wsplit);
+        const bool tc = dev >= 0 && dev < 256 && g_router_tc_ok[dev] && E % RT_BM == 0 && H % RT_BK == 0 &&
+                        L.wsplit + (size_t)3 * E * H * 2 <= L.total && tmap_bf16_rows(&tmA, planes, 3LL * E, H, RT_BM) &&
+                        tmap_bf16_rows(&tmB, x, T, H, RT_BN);
+        if (tc) {  // tensor cores: W_r as three exact bf16 planes, fp32 accumulation in TMEM
+            k_router_split<<<E, 256, 0, st>>>(W, E, H, planes, wnorm);
+            k_router_tc<<<dim3(E / RT_BM, (T + RT_BN - 1) / RT_BN), RT_THREADS, RT_SMEM, st>>>(tmA, tmB, T, H, E, b,
+                                                                                              logit);
+            ta.gfast = moe_tc_router_gamma(H);
+        } else {
+            k_router_norms<<<(E + 7) / 8, 256, 0, st>>>(W, E, H, wnorm);
+            k_router_gemm<<<dim3((E + RG_BN - 1) / RG_BN, (T + RG_BM - 1) / RG_BM), 256, 0, st>>>(x, T, H, W, b, E,
+                                                                                                  logit);
+            ta.gfast = gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);
+        }
         ta.wnorm = wnorm;
-        ta.gfast = gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);
-        k_topk<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+        float* xn = reinterpret_cast<float*>(ws + L.xn);
+        k_xnorm<<<(T + 7) / 8, 256, 0, st>>>(x, T, H, xn);
+        ta.xnorm = xn;
+        ta.slow_count = reinterpret_cast<int32_t*>(ws + L.slow);
+        ta.slow_list = ta.slow_count + 4;
+        if (cudaMemsetAsync(ta.slow_count, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+        k_topk_fast<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+        k_topk_slow<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     }
     PermArgs pa{};
     pa.idx = idx; pa.P = P; pa.E = E; pa.nchunks = (P + PERM_CHUNK - 1) / PERM_CHUNK;
@@ -148,7 +178,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
     k_perm_count<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
     k_perm_scan<<<1, MOE_MAX_E, 0, st>>>(pa);
     k_perm_scatter<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
-    count(T <= MOE_DECODE_MAX_T ? 5 : 6);
+    count(T <= MOE_DECODE_MAX_T ? 5 : 8);
     return cuda_rc(cudaGetLastError());
 }
 
@@ -166,6 +196,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     });
     return g_encode;
+}
+
+// bf16 [rows][K] row-major, box 64 x box_rows, 128-byte swizzle; rows past the end read as zero
+bool tmap_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+    if (!encoder()) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 [rows][K] row-major, box 64 x PF_BOX_ROWS, 128-byte swizzle
@@ -253,6 +295,7 @@ int ensure_init() {
     chk(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_decode_fused<4, 4, 16>, DF_THREADS, dfs));
     g_df_grid[dev] = (per >= 1) ? nsm : 0;
     g_df_maxdyn[dev] = dfs;
+    g_router_tc_ok[dev] = set_smem(k_router_tc, RT_SMEM) == cudaSuccess;
     if (e != cudaSuccess || !encoder()) return MOE_ERR_CUDA;
     g_init_mask[dev >> 6] |= 1ull << (dev & 63);
     return MOE_OK;
@@ -518,6 +561,7 @@ int moe_route(const uint16_t* x, int T, int H, const float* router_w, const floa
     if (T == 0) return MOE_OK;
     const Ws L = ws_layout(T, E, top_k, H, 32);
     if (ws_bytes < L.total) return MOE_ERR_WS;
+    if (T > MOE_DECODE_MAX_T && (rc = ensure_init()) != MOE_OK) return rc;  // the chunk router's kernel attributes
     return launch_route(x, T, H, router_w, router_bias, E, top_k, topk_idx, topk_w, expert_offsets, perm, nullptr,
                         static_cast<uint8_t*>(ws), L, false, nullptr, 0, static_cast<cudaStream_t>(stream));
 }

@@ -184,6 +184,8 @@ struct TopkArgs {
     int32_t* idx;           // [T][k]
     float* w;               // [T][k]
     int32_t* n_rechecked;   // [1]
+    int32_t* slow_list;     // tokens the fast pass could not certify (k_topk_fast), or null
+    int32_t* slow_count;    // [1] their number (zeroed before the fast pass)
     double gfast;           // gamma_n of the fast logits' summation
     int T, H, E, k;
 };
@@ -262,7 +264,10 @@ __device__ __forceinline__ void write_topk(int k, double cval, int ce, int32_t* 
 // MODE 0: fp32 logits, bound from norms (prefill); 1: fp64 logits with
 // per-entry sums of |x W| (decode kernels); 2: fp64 logits, bound from norms
 // (fused decode, whose router runs on the fp64 tensor cores).
-template <int MODE>
+// FAST_ONLY: a token whose fast values do not certify is appended to
+// a.slow_list (for k_topk_slow) instead of being finished here, which keeps the
+// fp64 re-evaluation's registers out of the common pass.
+template <int MODE, bool FAST_ONLY = false>
 __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* idx_out, float* w_out, int* cs,
                                            double* cvs, int32_t* nrechk) {
     constexpr bool F64 = MODE != 0;
@@ -419,6 +424,10 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         write_topk(k, cval, ce, idx_out, w_out);
         return;
     }
+    if (FAST_ONLY) {
+        if (lane == 0) a.slow_list[atomicAdd(a.slow_count, 1)] = t;
+        return;
+    }
     // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
     if (MODE == 0) {
         for (int base = 0; base < MC; base += 16) {
@@ -429,6 +438,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = ab[j] = 0.0;
             const uint16_t* xr = a.x + (size_t)t * H;
+#pragma unroll 4
             for (int h = lane; h < H; h += 32) {
                 const double xd = bf16_bits_to_f32(xr[h]);
 #pragma unroll
@@ -497,6 +507,50 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     }
     if (lane < k) w_out[lane] = (float)(mine / z);
     if (lane == 0 && nrechk) atomicAdd(nrechk, 1);
+}
+
+// ||x_t||_2 of every token, inflated to cover its fp32 rounding; one warp per token.
+__global__ void __launch_bounds__(256) k_xnorm(const uint16_t* __restrict__ x, int T, int H, float* __restrict__ xn) {
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    float s = 0.f;
+#pragma unroll 8
+    for (int i = lane; i < H / 8; i += 32) {
+        const uint4 r = __ldg(xr + i);
+        const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+            const float lo = __uint_as_float(wd[z] << 16), hi = __uint_as_float(wd[z] & 0xffff0000u);
+            s = fmaf(lo, lo, fmaf(hi, hi, s));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) xn[t] = sqrtf(s) * 1.001f;
+}
+
+// One warp per token: the fast pass; tokens it cannot certify go to k_topk_slow.
+template <int MODE>
+__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk_fast(TopkArgs a) {
+    __shared__ int s_ce[MOE_TOPK_WARPS][64];
+    __shared__ double s_cv[MOE_TOPK_WARPS][64];
+    const int wid = threadIdx.x >> 5;
+    const int t = blockIdx.x * MOE_TOPK_WARPS + wid;
+    if (t >= a.T) return;
+    topk_token<MODE, true>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
+}
+
+// The tokens k_topk_fast listed, one warp each (launched for up to T of them).
+template <int MODE>
+__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk_slow(TopkArgs a) {
+    __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
+    __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
+    const int wid = threadIdx.x >> 5;
+    const int i = blockIdx.x * MOE_TOPK_WARPS + wid;
+    if (i >= *a.slow_count) return;
+    const int t = a.slow_list[i];
+    topk_token<MODE>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
 }
 
 // One warp per token.

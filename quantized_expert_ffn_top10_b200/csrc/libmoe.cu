@@ -488,11 +488,13 @@ int run_decode(const LayerCall& c) {
     return cuda_rc(cudaGetLastError());
 }
 
+// mgroups CTAs per N-tile, each over mtiles / mgroups M-tiles (mgroups divides mtiles).
 template <int MODE, int B0, int B1>
-void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, const PrefillArgs& a,
-                 int mtiles, int ntile_max, cudaStream_t st) {
-    (void)mtiles;  // each CTA walks all M-tiles of its N-tile
-    k_prefill_gemm<MODE, B0, B1><<<ntile_max, PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
+void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, PrefillArgs a, int mtiles,
+                 int mgroups, int ntile_max, cudaStream_t st) {
+    while (mtiles % mgroups) --mgroups;
+    a.mgroups = mgroups;
+    k_prefill_gemm<MODE, B0, B1><<<ntile_max * mgroups, PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
 }
 
 int run_prefill(const LayerCall& c) {
@@ -525,14 +527,15 @@ int run_prefill(const LayerCall& c) {
     a.perm = r.perm; a.topk_w = r.w;
     const int nt = max_tiles(P, c.E);
     a.out = h;
-    if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, tg, tu, a, I / PF_BM, nt, c.st);
-    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
-    else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, tg, tu, a, I / PF_BM, nt, c.st);
-    else launch_gemm<0, 4, 2>(tx, tg, tu, a, I / PF_BM, nt, c.st);
+    const int mg1 = I / PF_BM, mg2 = std::max(1, H / PF_BM / 4);  // CTAs per N-tile: GEMM1 one per M-tile
+    if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
+    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
+    else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
+    else launch_gemm<0, 4, 2>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
     stage(2, c.st);
     a.out = y;
-    if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
-    else launch_gemm<1, 2, 2>(th, tdn, tdn, a, H / PF_BM, nt, c.st);
+    if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, tdn, tdn, a, H / PF_BM, mg2, nt, c.st);
+    else launch_gemm<1, 2, 2>(th, tdn, tdn, a, H / PF_BM, mg2, nt, c.st);
     stage(3, c.st);
     k_combine<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
         c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);

@@ -25,7 +25,7 @@
 
 #define PF_BK 64          // K elements per stage (one 128-byte swizzle row of bf16)
 #define PF_BM 128         // weight rows per M-tile
-#define PF_BN_MAX 256     // pair rows per tile
+#define PF_BN_MAX 256     // pair rows per tile (PREFILL_TILE_N)
 #define PF_BOX_ROWS 16    // activation rows per TMA box
 #define PF_EPI_WARP0 2    // epilogue warps 2..5 (TMEM lane quadrants 2, 3, 0, 1)
 #define PF_DQ_WARP0 6     // dequantisation warps 6..13
@@ -35,13 +35,16 @@
 template <int MODE>  // 0 = gate/up + SwiGLU, 1 = down + gate weight
 struct PfCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
-    static constexpr int STAGES = MODE == 0 ? 3 : 4;
+    static constexpr int TSTAGES = MODE == 0 ? 4 : 5;            // TMA ring: activation tile + raw codes
+    static constexpr int ASTAGES = 2;                            // ring of dequantised A tiles
     static constexpr int NACC = MODE == 0 ? 1 : 2;               // accumulator buffers in TMEM
+    static constexpr int MAT_COLS = PF_BN_MAX;                   // TMEM columns of one matrix's accumulator
+    static constexpr int ACC_COLS = NMAT * PF_BN_MAX;            // TMEM columns of one accumulator buffer
     static constexpr int A_BYTES = PF_BM * PF_BK * 2;            // one dequantised matrix tile
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int C_BYTES = PF_BM * PF_BK / 2;            // raw codes (<= 4-bit)
-    static constexpr int STAGE_BYTES = NMAT * A_BYTES + B_BYTES + NMAT * C_BYTES;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*gate weights*/ + 256 /*barriers*/;
+    static constexpr int SMEM = TSTAGES * (B_BYTES + NMAT * C_BYTES) + ASTAGES * NMAT * A_BYTES +
+                                1024 /*align*/ + 1024 /*gate weights*/ + 256 /*barriers*/;
     static constexpr int TMEM_COLS = 512;
 };
 
@@ -52,6 +55,7 @@ struct PrefillArgs {
     int64_t off_scales[3];
     int64_t slot_bytes;
     int H, I, E, k, layer;
+    int mgroups;             // CTAs per N-tile: each takes NOUT / PF_BM / mgroups consecutive M-tiles
     const int4* tiles;       // (expert, first pair row, rows, 0)
     const int32_t* meta;     // [1] = number of tiles
     const int32_t* perm;
@@ -132,28 +136,32 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     k_prefill_gemm(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC0,
                    const __grid_constant__ CUtensorMap tmC1, PrefillArgs a) {
     using C = PfCfg<MODE>;
-    const int tile = blockIdx.x;
+    // CTA b serves N-tile b / mgroups and its M-tile group b % mgroups: the CTAs
+    // sharing an activation tile are adjacent in launch order, so they run
+    // together and its re-reads are served by L2.
+    const int tile = blockIdx.x / a.mgroups, mgrp = blockIdx.x % a.mgroups;
     if (tile >= a.meta[1]) return;
     const int4 td = a.tiles[tile];
     const int e = td.x, row0 = td.y, nrows = td.z;
     const int npad = (nrows + 15) & ~15;
     const int K = MODE == 0 ? a.H : a.I;
     const int NOUT = MODE == 0 ? a.I : a.H;  // output features (row length of `out`)
-    const int nk = K / PF_BK, nmt = NOUT / PF_BM, nstage = nk * nmt;
+    const int nk = K / PF_BK, nmt = NOUT / PF_BM / a.mgroups, mt0 = mgrp * nmt, nstage = nk * nmt;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* sB = smem;                                          // [STAGES][B_BYTES]
-    uint8_t* sA = sB + C::STAGES * C::B_BYTES;                   // [STAGES][NMAT][A_BYTES]
-    uint8_t* sC = sA + C::STAGES * C::NMAT * C::A_BYTES;         // [STAGES][NMAT][C_BYTES]
-    float* s_w = reinterpret_cast<float*>(sC + C::STAGES * C::NMAT * C::C_BYTES);  // [256] gate weights
+    uint8_t* sB = smem;                                          // [TSTAGES][B_BYTES]
+    uint8_t* sC = sB + C::TSTAGES * C::B_BYTES;                  // [TSTAGES][NMAT][C_BYTES]
+    uint8_t* sA = sC + C::TSTAGES * C::NMAT * C::C_BYTES;        // [ASTAGES][NMAT][A_BYTES]
+    float* s_w = reinterpret_cast<float*>(sA + C::ASTAGES * C::NMAT * C::A_BYTES);  // [PF_BN_MAX] gate weights
     uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + PF_BN_MAX);
-    uint64_t* full = bars;                   // TMA bytes landed
-    uint64_t* deq = bars + C::STAGES;        // dequantised A written
-    uint64_t* empty = bars + 2 * C::STAGES;  // MMA finished reading the stage
-    uint64_t* accf = bars + 3 * C::STAGES;   // [NACC] accumulator final
-    uint64_t* acce = accf + C::NACC;         // [NACC] accumulator drained
+    uint64_t* full = bars;                      // [TSTAGES] TMA bytes landed
+    uint64_t* empty = full + C::TSTAGES;        // [TSTAGES] codes dequantised and activation tile consumed
+    uint64_t* deq = empty + C::TSTAGES;         // [ASTAGES] dequantised A written
+    uint64_t* aempty = deq + C::ASTAGES;        // [ASTAGES] MMA finished reading the A tile
+    uint64_t* accf = aempty + C::ASTAGES;       // [NACC] accumulator final
+    uint64_t* acce = accf + C::NACC;            // [NACC] accumulator drained
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + C::NACC);
 
     const int64_t slot = a.slot_table[(int64_t)a.layer * a.E + e];
@@ -165,10 +173,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < C::TSTAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&empty[s], PF_DQ_THREADS / 32 + 1);  // every dequant warp, and the MMA commit
+        }
+        for (int s = 0; s < C::ASTAGES; ++s) {
             mbar_init(&deq[s], PF_DQ_THREADS / 32);
-            mbar_init(&empty[s], 1);
+            mbar_init(&aempty[s], 1);
         }
         for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&accf[b], 1);
@@ -195,8 +206,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (C::NMAT == 2) tma_prefetch_desc(&tmC1);
             const uint32_t bytes = npad * PF_BK * 2 + PF_BM * PF_BK * B0 / 8 + (C::NMAT == 2 ? PF_BM * PF_BK * B1 / 8 : 0);
             for (int i = 0; i < nstage && alive; ++i) {
-                const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
-                const int kb = i % nk, rowbase = (i / nk) * PF_BM;
+                const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
+                const int kb = i % nk, rowbase = (mt0 + i / nk) * PF_BM;
                 if (!mbar_wait(&empty[s], ph ^ 1)) { alive = false; break; }
                 mbar_arrive_expect_tx(&full[s], bytes);
                 for (int r = 0; r < npad; r += PF_BOX_ROWS)
@@ -221,11 +232,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int buf = mt % C::NACC, use = mt / C::NACC;
                 if (!mbar_wait(&acce[buf], (use & 1) ^ 1)) { alive = false; break; }  // drained by the epilogue
                 tc_fence_after();
-                const uint32_t dcol = tmem + buf * 256;
+                const uint32_t dcol = tmem + buf * C::ACC_COLS;
                 for (int kb = 0; kb < nk; ++kb) {
                     const int i = mt * nk + kb;
-                    const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
-                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&deq[s], ph)) { alive = false; break; }
+                    const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
+                    const int sa = i % C::ASTAGES, pa = (i / C::ASTAGES) & 1;
+                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&deq[sa], pa)) { alive = false; break; }
                     tc_fence_after();
                     const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
@@ -233,11 +245,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const uint64_t bdesc = make_sdesc_sw128(bb + kk * 32);
 #pragma unroll
                         for (int m = 0; m < C::NMAT; ++m) {
-                            const uint32_t ab = smem_u32(sA + (s * C::NMAT + m) * C::A_BYTES);
-                            tc_mma_bf16(dcol + m * 256, make_sdesc_sw128(ab + kk * 32), bdesc, idesc, (kb | kk) != 0);
+                            const uint32_t ab = smem_u32(sA + (sa * C::NMAT + m) * C::A_BYTES);
+                            tc_mma_bf16(dcol + m * C::MAT_COLS, make_sdesc_sw128(ab + kk * 32), bdesc, idesc,
+                                        (kb | kk) != 0);
                         }
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit(&empty[s]);    // the activation tile may be refilled
+                    tc_commit(&aempty[sa]);  // the A tile may be rewritten
                 }
                 tc_commit(&accf[buf]);
             }
@@ -248,21 +262,56 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const uint8_t* sbase = a.arena + slot * a.slot_bytes;
         const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[MODE == 0 ? 0 : 2]);
         const uint16_t* sc1 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[1]);
+        // One 16-byte load holds this thread's scales for 4 consecutive stages (blocks
+        // 2 kb .. 2 kb + 7 of its row); when nk % 4 == 0 groups of 4 stages never
+        // straddle an M-tile and the next group's scales are loaded a group ahead.
+        // Otherwise (K % 256 != 0) each stage loads its own scale.
+        const bool grouped = (nk & 3) == 0;
+        const int ngrp = grouped ? nstage / 4 : 0;
+        auto load_grp = [&](int gi, uint4& r0, uint4& r1) {
+            const int i0 = gi * 4, kb0 = i0 % nk;
+            const size_t base = (size_t)((mt0 + i0 / nk) * PF_BM + row) * (K / 32) + 2 * kb0;
+            r0 = __ldg(reinterpret_cast<const uint4*>(sc0 + base));
+            if (C::NMAT == 2) r1 = __ldg(reinterpret_cast<const uint4*>(sc1 + base));
+        };
+        auto pick = [](const uint4& v, int idx) -> uint16_t {  // half idx (0..7) of v
+            const int wi = idx >> 1;
+            const uint32_t w = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
+            return (uint16_t)(w >> (16 * (idx & 1)));
+        };
+        uint4 cur0 = make_uint4(0, 0, 0, 0), cur1 = cur0, nxt0 = cur0, nxt1 = cur0;
+        if (ngrp > 0) load_grp(0, cur0, cur1);
+        if (ngrp > 1) load_grp(1, nxt0, nxt1);
         for (int i = 0; i < nstage; ++i) {
-            const int s = i % C::STAGES, ph = (i / C::STAGES) & 1;
-            const int kb = i % nk;
-            const size_t grow = (size_t)((i / nk) * PF_BM + row);  // weight row in the matrix
-            const uint16_t q0 = __ldg(sc0 + grow * (K / 32) + 2 * kb + half);
-            const uint16_t q1 = C::NMAT == 2 ? __ldg(sc1 + grow * (K / 32) + 2 * kb + half) : 0;
-            if (!mbar_wait(&full[s], ph)) { alive = false; break; }
-            dequant_unit<B0>(sC + (s * C::NMAT + 0) * C::C_BYTES, sA + (s * C::NMAT + 0) * C::A_BYTES, row, half,
+            const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
+            const int sa = i % C::ASTAGES, pa = (i / C::ASTAGES) & 1;
+            uint16_t q0, q1 = 0;
+            if (grouped) {
+                if ((i & 3) == 0 && i > 0) {
+                    cur0 = nxt0;
+                    cur1 = nxt1;
+                    if ((i >> 2) + 1 < ngrp) load_grp((i >> 2) + 1, nxt0, nxt1);
+                }
+                const int si = 2 * (i & 3) + half;
+                q0 = pick(cur0, si);
+                if (C::NMAT == 2) q1 = pick(cur1, si);
+            } else {
+                const size_t grow = (size_t)((mt0 + i / nk) * PF_BM + row);  // weight row in the matrix
+                q0 = __ldg(sc0 + grow * (K / 32) + 2 * (i % nk) + half);
+                if (C::NMAT == 2) q1 = __ldg(sc1 + grow * (K / 32) + 2 * (i % nk) + half);
+            }
+            if (!mbar_wait(&full[s], ph) || !mbar_wait(&aempty[sa], pa ^ 1)) { alive = false; break; }
+            dequant_unit<B0>(sC + (s * C::NMAT + 0) * C::C_BYTES, sA + (sa * C::NMAT + 0) * C::A_BYTES, row, half,
                              half_bits_to_f32(q0));
             if (C::NMAT == 2)
-                dequant_unit<B1>(sC + (s * C::NMAT + 1) * C::C_BYTES, sA + (s * C::NMAT + 1) * C::A_BYTES, row, half,
-                                 half_bits_to_f32(q1));
+                dequant_unit<B1>(sC + (s * C::NMAT + 1) * C::C_BYTES, sA + (sa * C::NMAT + 1) * C::A_BYTES, row,
+                                 half, half_bits_to_f32(q1));
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&deq[s]);
+            if (lane == 0) {
+                mbar_arrive(&deq[sa]);
+                mbar_arrive(&empty[s]);  // this warp's reads of the codes are done
+            }
         }
     } else {  // epilogue warps: TMEM -> registers -> global, one M-tile at a time
         const int q = warp & 3;  // TMEM lane quadrant this warp may read
@@ -270,12 +319,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const int buf = mt % C::NACC, use = mt / C::NACC;
             if (!mbar_wait(&accf[buf], use & 1)) { alive = false; break; }
             tc_fence_after();
-            const int r = mt * PF_BM + q * 32 + lane;  // output feature of this thread
-            const uint32_t ta0 = tmem + buf * 256 + ((uint32_t)(q * 32) << 16);
+            const int r = (mt0 + mt) * PF_BM + q * 32 + lane;  // output feature of this thread
+            const uint32_t ta0 = tmem + buf * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
             for (int c0 = 0; c0 < npad; c0 += 16) {
                 uint32_t v0[16], v1[16];
                 tmem_ld16(ta0 + c0, v0);
-                if (MODE == 0) tmem_ld16(ta0 + 256 + c0, v1);
+                if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0, v1);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {

@@ -46,7 +46,7 @@
 #define DF_MAXP 256        // pairs T * k
 #define DF_FT 16           // features per phase-D tile
 #define DF_MAX_EPC 8       // router experts per CTA (rows of the fp64 MMA)
-#define DF_MAX_NBD 16      // quant blocks of a W_d row (I <= 512 at 4 bits)
+#define DF_MAX_NBD 16      // quant blocks of a W_d row (I <= 512)
 #define DF_SMEM_LIMIT (227 * 1024)
 #define DF_BAR_WORDS (32 * 18)  // grid barrier: 16 group counters, the top counter, the flag
 #define DF_NREP 8          // copies of the (logit, bound) records that phase B reads
@@ -510,80 +510,14 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
 
 // ---------------------------------------------------------------- phase D: one expert, one feature tile
 
-// W_d rows ft .. ft + 15 (all I columns: nblk = I / 32 <= 16 blocks) and scales.
-struct DfDRegs {
-    uint32_t c0[DF_MAX_NBD], c1[DF_MAX_NBD];
-    uint4 s0[DF_MAX_NBD / 8], s1[DF_MAX_NBD / 8];
-};
-
-// The unit's codes sit as [16 rows][nbox 128-byte chunks] with the TMA
-// 128-byte swizzle keyed on the 128-byte line index (row * nbox + chunk).
-template <int BD, int nblk>
-__device__ __forceinline__ void df_stage_d(const uint8_t* code, const uint8_t* sc, DfDRegs& r) {
-    constexpr int nbox = nblk * BD / 32;
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, key16 = (g & 7) << 4;
-    if (BD == 4) {
-        // blocks j, j + 1 of rows 0-7 / 8-15: matrices (rows 0-7, j), (8-15, j), (0-7, j+1), (8-15, j+1)
-        const int row = ((lane >> 3) & 1) * 8 + (lane & 7), jo = lane >> 4;
-#pragma unroll
-        for (int j = 0; j < DF_MAX_NBD; j += 2) {
-            if (j < nblk) {
-                const int jj = j + jo, line = row * nbox + (jj >> 3);
-                ldsm_x4(code + line * 128 + (((jj & 7) ^ (line & 7)) << 4), r.c0[j], r.c1[j], r.c0[j + 1], r.c1[j + 1]);
-            } else {
-                r.c0[j] = r.c1[j] = r.c0[j + 1] = r.c1[j + 1] = 0u;
-            }
-        }
-    } else {  // 2 bits: one 128-byte chunk per row (nbox == 1), the gate/up layout
-        const uint8_t* r0 = code + g * 128;
-#pragma unroll
-        for (int j = 0; j < DF_MAX_NBD; ++j) {
-            r.c0[j] = j < nblk ? ld_codes<BD>(r0, j, q, key16) : 0u;
-            r.c1[j] = j < nblk ? ld_codes<BD>(r0 + 1024, j, q, key16) : 0u;
-        }
-    }
-    constexpr int ns = nblk / 8;  // uint4 of scales per row
-#pragma unroll
-    for (int i = 0; i < DF_MAX_NBD / 8; ++i) {
-        r.s0[i] = i < ns ? *reinterpret_cast<const uint4*>(sc + (g * ns + i) * 16) : make_uint4(0u, 0u, 0u, 0u);
-        r.s1[i] = i < ns ? *reinterpret_cast<const uint4*>(sc + ((g + 8) * ns + i) * 16) : make_uint4(0u, 0u, 0u, 0u);
-    }
-}
-
-// acc (features g, g + 8; pair columns 2q, 2q + 1) = W_d rows x h of the
-// expert's n pairs.  hs: staged h of the first pair [n][hstride bytes], in
-// fragment order; hsum: per pair and block, the sum of its 32 h values.
-template <int BD, int nblk>
-__device__ __forceinline__ void df_compute_d(const DfDRegs& r, const uint8_t* hs, int hstride, const float* hsum,
-                                             int n, float (&acc)[4]) {
-    constexpr float kOff = 128.f + (float)(1 << (BD - 1));
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const bool col_ok = g < n, ok0 = 2 * q < n, ok1 = 2 * q + 1 < n;
-#pragma unroll
-    for (int j = 0; j < DF_MAX_NBD; ++j) {
-        if (j < nblk) {
-            uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-            if (col_ok) bx = *reinterpret_cast<const uint4*>(hs + g * hstride + j * 64 + q * 16);
-            const float h0 = ok0 ? hsum[(2 * q) * nblk + j] : 0.f;
-            const float h1 = ok1 ? hsum[(2 * q + 1) * nblk + j] : 0.f;
-            uint32_t p0[4], p1[4];
-            unpack8<BD>(r.c0[j], p0);
-            unpack8<BD>(r.c1[j], p1);
-            float d[4] = {-kOff * h0, -kOff * h1, -kOff * h0, -kOff * h1};
-            mma_bf16_16816(d, p0[0], p1[0], p0[1], p1[1], bx.x, bx.y);
-            mma_bf16_16816(d, p0[2], p1[2], p0[3], p1[3], bx.z, bx.w);
-            const float s0 = df_scale(r.s0, j), s1 = df_scale(r.s1, j);
-            acc[0] = fmaf(s0, d[0], acc[0]);
-            acc[1] = fmaf(s0, d[1], acc[1]);
-            acc[2] = fmaf(s1, d[2], acc[2]);
-            acc[3] = fmaf(s1, d[3], acc[3]);
-        }
-    }
-}
-
-// The same product computed straight from the slot in a rolled loop (two
+// acc (features g, g + 8; pair columns 2q, 2q + 1) = W_d rows ft .. ft + 15 x h
+// of the expert's n pairs, straight from the slot in a rolled loop (two
 // blocks per step): a W_d unit is used once per launch, so its code stays
-// small instead of being unrolled over all blocks.
+// small instead of being unrolled over all blocks.  The unit's codes sit as
+// [16 rows][nbox 128-byte chunks] with the TMA 128-byte swizzle keyed on the
+// 128-byte line index (row * nbox + chunk); scales as [16 rows][nblk] fp16;
+// hs: h of the first pair [n][hstride bytes] in fragment order; hsum: per pair
+// and block, the sum of its 32 h values.
 template <int BD, int nblk>
 __device__ __forceinline__ void df_compute_d_smem(const uint8_t* code, const uint8_t* sc, const uint8_t* hs, int hstride,
                                                   const float* hsum, int n, float (&acc)[4]) {

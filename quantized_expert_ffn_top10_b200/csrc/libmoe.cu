@@ -210,29 +210,6 @@ bool tmap_bf16_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K, i
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [rows][K] row-major, box 64 x PF_BOX_ROWS, 128-byte swizzle
-bool tmap_act(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {PF_BK, PF_BOX_ROWS};
-    cuuint32_t es[2] = {1, 1};
-    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// codes of one matrix across all slots: uint8 [n_slots][rows][row_bytes], box (PF_BK*bits/8) x 128 x 1
-bool tmap_codes(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes, int64_t n_slots,
-                int64_t slot_bytes, int bits) {
-    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_slots};
-    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)slot_bytes};
-    cuuint32_t box[3] = {(cuuint32_t)(PF_BK * bits / 8), PF_BM, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Gate and up codes of every slot as one 5-D tensor: (128-byte chunk, chunk
 // index, row, matrix, slot); a box is 16 rows x one chunk of both matrices,
 // landing as [matrix][row][128 B] with the 128-byte swizzle.
@@ -488,13 +465,22 @@ int run_decode(const LayerCall& c) {
     return cuda_rc(cudaGetLastError());
 }
 
+// The activation matrix [rows][K] bf16 seen through boxes of 128, 64, 32 and 16 rows.
+struct ActMaps {
+    CUtensorMap m[4];
+    bool make(const void* base, int64_t rows, int64_t K) {
+        return tmap_bf16_rows(&m[0], base, rows, K, 128) && tmap_bf16_rows(&m[1], base, rows, K, 64) &&
+               tmap_bf16_rows(&m[2], base, rows, K, 32) && tmap_bf16_rows(&m[3], base, rows, K, 16);
+    }
+};
+
 // mgroups CTAs per N-tile, each over mtiles / mgroups M-tiles (mgroups divides mtiles).
 template <int MODE, int B0, int B1>
-void launch_gemm(const CUtensorMap& tb, const CUtensorMap& tc0, const CUtensorMap& tc1, PrefillArgs a, int mtiles,
-                 int mgroups, int ntile_max, cudaStream_t st) {
+void launch_gemm(const ActMaps& t, PrefillArgs a, int mtiles, int mgroups, int ntile_max, cudaStream_t st) {
     while (mtiles % mgroups) --mgroups;
     a.mgroups = mgroups;
-    k_prefill_gemm<MODE, B0, B1><<<ntile_max * mgroups, PF_THREADS, PfCfg<MODE>::SMEM, st>>>(tb, tc0, tc1, a);
+    k_prefill_gemm<MODE, B0, B1><<<ntile_max * mgroups, PF_THREADS, PfCfg<MODE>::SMEM, st>>>(t.m[0], t.m[1], t.m[2],
+                                                                                             t.m[3], a);
 }
 
 int run_prefill(const LayerCall& c) {
@@ -511,16 +497,12 @@ int run_prefill(const LayerCall& c) {
     uint16_t* h = reinterpret_cast<uint16_t*>(c.ws + L.h);
     uint16_t* y = reinterpret_cast<uint16_t*>(c.ws + L.y);
     k_gather_rows<<<P, 128, 0, c.st>>>(c.x, r.perm, P, H, c.k, xp);
-    CUtensorMap tx, th, tg, tu, tdn;
+    ActMaps tx, th;
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
-    if (!tmap_act(&tx, xp, P, H) || !tmap_act(&th, h, P, I) ||
-        !tmap_codes(&tg, c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8, ns, sb, d->bits_gate) ||
-        !tmap_codes(&tu, c.arena + d->off_codes[1], I, (int64_t)H * d->bits_up / 8, ns, sb, d->bits_up) ||
-        !tmap_codes(&tdn, c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb, d->bits_down))
-        return MOE_ERR_CUDA;
+    if (!tx.make(xp, P, H) || !th.make(h, P, I)) return MOE_ERR_CUDA;
     PrefillArgs a{};
     a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = ns; a.slot_bytes = sb;
-    for (int m = 0; m < 3; ++m) a.off_scales[m] = d->off_scales[m];
+    for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
     a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer;
     a.tiles = reinterpret_cast<const int4*>(c.ws + L.tiles);
     a.meta = reinterpret_cast<const int32_t*>(c.ws + L.meta);
@@ -529,14 +511,14 @@ int run_prefill(const LayerCall& c) {
     a.out = h;
     // CTAs per N-tile (measured best at H = 2048, I = 512: two each, GEMM1 over 2 M-tiles, GEMM2 over 8)
     const int mg1 = std::max(1, I / PF_BM / 2), mg2 = std::max(1, H / PF_BM / 8);
-    if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
-    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
-    else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
-    else launch_gemm<0, 4, 2>(tx, tg, tu, a, I / PF_BM, mg1, nt, c.st);
+    if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, a, I / PF_BM, mg1, nt, c.st);
+    else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, a, I / PF_BM, mg1, nt, c.st);
+    else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, a, I / PF_BM, mg1, nt, c.st);
+    else launch_gemm<0, 4, 2>(tx, a, I / PF_BM, mg1, nt, c.st);
     stage(2, c.st);
     a.out = y;
-    if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, tdn, tdn, a, H / PF_BM, mg2, nt, c.st);
-    else launch_gemm<1, 2, 2>(th, tdn, tdn, a, H / PF_BM, mg2, nt, c.st);
+    if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, a, H / PF_BM, mg2, nt, c.st);
+    else launch_gemm<1, 2, 2>(th, a, H / PF_BM, mg2, nt, c.st);
     stage(3, c.st);
     k_combine<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
         c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);

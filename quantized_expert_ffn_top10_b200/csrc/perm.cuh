@@ -11,7 +11,7 @@
 #include "common.cuh"
 
 #define PERM_CHUNK 1024
-#define PREFILL_TILE_N 256  // max tokens per grouped-GEMM tile
+#define PREFILL_TILE_N 192  // max tokens per grouped-GEMM tile
 
 struct PermArgs {
     const int32_t* idx;   // [P]

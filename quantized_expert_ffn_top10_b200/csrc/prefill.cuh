@@ -1,7 +1,7 @@
 // Prefill path: per-expert grouped GEMMs on the 5th-generation tensor cores.
 //
 // Rows of the grouped activation matrix follow the expert-sorted pair order
-// (perm).  A tile is (expert e, up to 256 consecutive pair rows of e, 128
+// (perm).  A tile is (expert e, up to 192 consecutive pair rows of e, 128
 // output features).  The MMA runs "weights x activations": the 128 weight rows
 // are the M side, the tile's pair rows the N side (N = rows rounded up to 16),
 // so a lightly loaded expert wastes at most 15 columns.
@@ -11,47 +11,66 @@
 //   GEMM2: D = W_d[rows] h^T                           (K = I)
 //          Y[pair][row] = bf16(w_pair * D)
 //
-// A CTA owns one N-tile and walks all M-tiles, so the activation rows stay in
-// L2 and setup is paid once.  Roles (448 threads): warp 0 issues TMA loads of
-// the activation tile (128-B swizzled) and of the raw code tile of each weight
-// matrix (one 3-D tensor map spans all arena slots); warp 1 owns TMEM and one
-// of its threads issues tcgen05.mma; warps 2-5 drain finished accumulators
-// (TMEM -> registers -> global; the down GEMM double-buffers them so this
-// overlaps the next M-tile); warps 6-13 dequantise codes to bf16 straight into
-// the 128-B swizzled K-major layout the MMA reads.  Stages cycle through full /
-// dequantised / empty mbarriers; every wait is bounded.
+// The dequantised weights never touch shared memory: they are written to
+// tensor memory (tcgen05.st) and the MMA takes its A operand from there, so
+// shared memory holds only the activation tiles and the tensor core reads
+// only B from it.  TMEM (512 columns): the accumulators (gate and up for
+// GEMM1, two buffers for GEMM2, PF_BN_MAX columns each) and, above them, a
+// ring of A slots, each K = 32 of every weight matrix (16 columns per matrix).
+//
+// A CTA owns one N-tile and walks its M-tiles, so the activation rows stay in
+// L2 and setup is paid once.  Roles (448 threads): warp 0 issues the TMA loads
+// of the activation tile (128-B swizzled K-major; a tile of npad rows goes as
+// at most one box each of 128, 64, 32 and 16 rows, since the TMA engine's cost
+// grows with the number of boxes); warp 1 owns TMEM and one of its threads
+// issues tcgen05.mma (GEMM1: for the gate matrix, while a thread of warp 22
+// issues the up matrix's: one thread issues at most one MMA per ~100 cycles,
+// about 80 cycles of tensor work at N = 160); warps 2-5 drain finished accumulators (TMEM -> registers
+// -> global; the down GEMM double-buffers them so this
+// overlaps the next M-tile); warps 6-21 load their own codes and scales from
+// the arena, PF_PREFETCH stages ahead in registers, and dequantise them into
+// the A slots (one 32-element block of 32 rows per warp and stage).  Rings: full / empty (activation tiles) and dequantised / free
+// (A slots) mbarriers; every wait is bounded.
 #pragma once
 #include "common.cuh"
 
 #define PF_BK 64          // K elements per stage (one 128-byte swizzle row of bf16)
+#define PF_AK 32          // K elements per A slot (one quantisation block)
 #define PF_BM 128         // weight rows per M-tile
-#define PF_BN_MAX 256     // pair rows per tile (PREFILL_TILE_N)
-#define PF_BOX_ROWS 16    // activation rows per TMA box
+#define PF_BN_MAX 192     // pair rows per tile (PREFILL_TILE_N)
 #define PF_EPI_WARP0 2    // epilogue warps 2..5 (TMEM lane quadrants 2, 3, 0, 1)
-#define PF_DQ_WARP0 6     // dequantisation warps 6..13
-#define PF_DQ_THREADS 256
-#define PF_THREADS 448
+#define PF_DQ_WARP0 6     // dequantisation warps 6..21 (four per TMEM lane quadrant)
+#define PF_DQ_THREADS 512
+#define PF_MMA2_WARP 22   // second MMA-issuing warp (GEMM1 up matrix)
+#define PF_THREADS 736
+#define PF_PREFETCH 4     // stages of codes and scales a dequantising thread holds ahead
 
 template <int MODE>  // 0 = gate/up + SwiGLU, 1 = down + gate weight
 struct PfCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;
-    static constexpr int TSTAGES = MODE == 0 ? 4 : 5;            // TMA ring: activation tile + raw codes
-    static constexpr int ASTAGES = 2;                            // ring of dequantised A tiles
+    static constexpr int TSTAGES = 6;                            // ring of activation tiles
     static constexpr int NACC = MODE == 0 ? 1 : 2;               // accumulator buffers in TMEM
     static constexpr int MAT_COLS = PF_BN_MAX;                   // TMEM columns of one matrix's accumulator
     static constexpr int ACC_COLS = NMAT * PF_BN_MAX;            // TMEM columns of one accumulator buffer
-    static constexpr int A_BYTES = PF_BM * PF_BK * 2;            // one dequantised matrix tile
-    static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
-    static constexpr int C_BYTES = PF_BM * PF_BK / 2;            // raw codes (<= 4-bit)
-    static constexpr int SMEM = TSTAGES * (B_BYTES + NMAT * C_BYTES) + ASTAGES * NMAT * A_BYTES +
-                                1024 /*align*/ + 1024 /*gate weights*/ + 256 /*barriers*/;
+    static constexpr int A_COL0 = NACC * ACC_COLS;               // first TMEM column of the A slots
+    static constexpr int SLOT_COLS = NMAT * (PF_AK / 2);         // TMEM columns of one A slot
     static constexpr int TMEM_COLS = 512;
+    static constexpr int ASLOTS = (TMEM_COLS - A_COL0) / SLOT_COLS;  // 4 (GEMM1) or 8 (GEMM2)
+    static constexpr int NISSUE = NMAT;                          // MMA-issuing threads, one per matrix
+    // A-slot arrivals per matrix: the four dequant warps (one per TMEM lane quadrant) writing it
+    static constexpr int DQ_ARRIVALS = 4;
+    static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
+    static_assert(A_COL0 + ASLOTS * SLOT_COLS <= TMEM_COLS && ASLOTS >= 4, "TMEM budget");
+    static_assert((2 * TSTAGES + 2 * NMAT * ASLOTS + 2 * NACC) * 8 + 4 <= BAR_BYTES, "barrier area");
 };
 
 struct PrefillArgs {
     const uint8_t* arena;
     const int32_t* slot_table;
     int64_t n_slots;
+    int64_t off_codes[3];
     int64_t off_scales[3];
     int64_t slot_bytes;
     int H, I, E, k, layer;
@@ -104,37 +123,42 @@ __device__ __forceinline__ uint4 dq8(uint32_t w, uint32_t s2hi, uint32_t s2lo) {
     return r;
 }
 
-// One 32-element block of one row: codes from the staging tile -> 4 swizzled
-// 16-byte chunks of the A tile (row r at r * 128 B, chunk j at (j ^ (r & 7)) * 16).
+// Codes of one 32-element block of one row: 16 bytes (4-bit) or 8 (2-bit, in .x and .y).
 template <int BITS>
-__device__ __forceinline__ void dequant_unit(const uint8_t* ctile, uint8_t* atile, int row, int half, float s) {
-    constexpr int ROWB = PF_BK * BITS / 8;  // staged code bytes per row
-    const uint8_t* src = ctile + row * ROWB + half * (32 * BITS / 8);
+__device__ __forceinline__ uint4 load_block_codes(const uint8_t* p) {
+    if (BITS == 4) return __ldg(reinterpret_cast<const uint4*>(p));
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    return make_uint4(v.x, v.y, 0u, 0u);
+}
+
+// One 32-element block of one row, codes in registers -> 16 columns of bf16
+// pairs (elements 2c, 2c + 1 in column c), the TMEM layout of an A row.
+template <int BITS>
+__device__ __forceinline__ void dequant_block_cols(uint4 c, float s, uint32_t (&col)[16]) {
     uint32_t w[4];
     if (BITS == 4) {
-        uint4 v = *reinterpret_cast<const uint4*>(src);
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        w[0] = c.x; w[1] = c.y; w[2] = c.z; w[3] = c.w;
     } else {
-        uint2 v = *reinterpret_cast<const uint2*>(src);
-        w[0] = v.x & 0xffffu; w[1] = v.x >> 16; w[2] = v.y & 0xffffu; w[3] = v.y >> 16;
+        w[0] = c.x & 0xffffu; w[1] = c.x >> 16; w[2] = c.y & 0xffffu; w[3] = c.y >> 16;
     }
     const float shi = __bfloat162float(__float2bfloat16_rn(s));
     const uint32_t s2hi = pack_bf16x2(shi, shi), s2lo = pack_bf16x2(s - shi, s - shi);  // both exact
-    uint8_t* rowp = atile + row * 128;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {  // chunk cc holds elements 8cc..8cc+7 of this block
-        const int j = half * 4 + cc;
-        *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = dq8<BITS>(w[cc], s2hi, s2lo);
+    for (int cc = 0; cc < 4; ++cc) {  // elements 8cc..8cc+7 -> columns 4cc..4cc+3
+        const uint4 v = dq8<BITS>(w[cc], s2hi, s2lo);
+        col[4 * cc + 0] = v.x; col[4 * cc + 1] = v.y; col[4 * cc + 2] = v.z; col[4 * cc + 3] = v.w;
     }
 }
 
-// One CTA per N-tile (expert e, rows row0 .. row0+nrows of the grouped
-// activations); it walks every M-tile of the output features.  Stage i covers
-// (M-tile i / nk, K-block i % nk).
+// One CTA per (N-tile, M-tile group): expert e, rows row0 .. row0+nrows of the
+// grouped activations, M-tiles mt0 .. mt0+nmt of the output features.  Stage i
+// covers (M-tile mt0 + i / nk, K-block i % nk) and A slots 2i, 2i + 1 (its two
+// halves).  The four tensor maps view the same activation matrix with boxes of
+// 128, 64, 32 and 16 rows.
 template <int MODE, int B0, int B1>
 __global__ void __launch_bounds__(PF_THREADS, 1)
-    k_prefill_gemm(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC0,
-                   const __grid_constant__ CUtensorMap tmC1, PrefillArgs a) {
+    k_prefill_gemm(const __grid_constant__ CUtensorMap tx128, const __grid_constant__ CUtensorMap tx64,
+                   const __grid_constant__ CUtensorMap tx32, const __grid_constant__ CUtensorMap tx16, PrefillArgs a) {
     using C = PfCfg<MODE>;
     // CTA b serves N-tile b / mgroups and its M-tile group b % mgroups: the CTAs
     // sharing an activation tile are adjacent in launch order, so they run
@@ -151,16 +175,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* sB = smem;                                          // [TSTAGES][B_BYTES]
-    uint8_t* sC = sB + C::TSTAGES * C::B_BYTES;                  // [TSTAGES][NMAT][C_BYTES]
-    uint8_t* sA = sC + C::TSTAGES * C::NMAT * C::C_BYTES;        // [ASTAGES][NMAT][A_BYTES]
-    float* s_w = reinterpret_cast<float*>(sA + C::ASTAGES * C::NMAT * C::A_BYTES);  // [PF_BN_MAX] gate weights
+    uint8_t* sB = smem;                                            // [TSTAGES][B_BYTES]
+    float* s_w = reinterpret_cast<float*>(sB + C::TSTAGES * C::B_BYTES);  // [PF_BN_MAX] gate weights
     uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + PF_BN_MAX);
-    uint64_t* full = bars;                      // [TSTAGES] TMA bytes landed
-    uint64_t* empty = full + C::TSTAGES;        // [TSTAGES] codes dequantised and activation tile consumed
-    uint64_t* deq = empty + C::TSTAGES;         // [ASTAGES] dequantised A written
-    uint64_t* aempty = deq + C::ASTAGES;        // [ASTAGES] MMA finished reading the A tile
-    uint64_t* accf = aempty + C::ASTAGES;       // [NACC] accumulator final
+    uint64_t* full = bars;                      // [TSTAGES] activation tile landed
+    uint64_t* empty = full + C::TSTAGES;        // [TSTAGES] MMA done reading the activation tile
+    uint64_t* deq = empty + C::TSTAGES;         // [NMAT][ASLOTS] A slot of a matrix written
+    uint64_t* aempty = deq + C::NMAT * C::ASLOTS;  // [NMAT][ASLOTS] MMA done reading it
+    uint64_t* accf = aempty + C::NMAT * C::ASLOTS;  // [NACC] accumulator final
     uint64_t* acce = accf + C::NACC;            // [NACC] accumulator drained
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + C::NACC);
 
@@ -175,14 +197,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::TSTAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], PF_DQ_THREADS / 32 + 1);  // every dequant warp, and the MMA commit
+            mbar_init(&empty[s], C::NISSUE);
         }
-        for (int s = 0; s < C::ASTAGES; ++s) {
-            mbar_init(&deq[s], PF_DQ_THREADS / 32);
+        for (int s = 0; s < C::NMAT * C::ASLOTS; ++s) {
+            mbar_init(&deq[s], C::DQ_ARRIVALS);
             mbar_init(&aempty[s], 1);
         }
         for (int b = 0; b < C::NACC; ++b) {
-            mbar_init(&accf[b], 1);
+            mbar_init(&accf[b], C::NISSUE);
             mbar_init(&acce[b], 4);
         }
         fence_mbar_init();
@@ -201,140 +223,174 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&tmB);
-            tma_prefetch_desc(&tmC0);
-            if (C::NMAT == 2) tma_prefetch_desc(&tmC1);
-            const uint32_t bytes = npad * PF_BK * 2 + PF_BM * PF_BK * B0 / 8 + (C::NMAT == 2 ? PF_BM * PF_BK * B1 / 8 : 0);
-            for (int i = 0; i < nstage && alive; ++i) {
+            tma_prefetch_desc(&tx128);
+            tma_prefetch_desc(&tx64);
+            tma_prefetch_desc(&tx32);
+            tma_prefetch_desc(&tx16);
+            const uint32_t bytes = npad * PF_BK * 2;
+            for (int i = 0; i < nstage; ++i) {
                 const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-                const int kb = i % nk, rowbase = (mt0 + i / nk) * PF_BM;
-                if (!mbar_wait(&empty[s], ph ^ 1)) { alive = false; break; }
+                const int kc = (i % nk) * PF_BK;
+                if (!mbar_wait_fast(&empty[s], ph ^ 1)) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
-                for (int r = 0; r < npad; r += PF_BOX_ROWS)
-                    tma_load_2d(sB + s * C::B_BYTES + r * 128, &tmB, &full[s], kb * PF_BK, row0 + r);
-                asm volatile(
-                    "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
-                        "r"(smem_u32(sC + (s * C::NMAT + 0) * C::C_BYTES)), "l"(&tmC0), "r"(smem_u32(&full[s])),
-                    "r"(kb * PF_BK * B0 / 8), "r"(rowbase), "r"((int)slot)
-                    : "memory");
-                if (C::NMAT == 2)
-                    asm volatile(
-                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
-                            "r"(smem_u32(sC + (s * C::NMAT + 1) * C::C_BYTES)), "l"(&tmC1), "r"(smem_u32(&full[s])),
-                        "r"(kb * PF_BK * B1 / 8), "r"(rowbase), "r"((int)slot)
-                        : "memory");
+                uint8_t* dst = sB + s * C::B_BYTES;  // row r at r * 128 B
+                int r = 0;
+                for (; r + 128 <= npad; r += 128) tma_load_2d(dst + r * 128, &tx128, &full[s], kc, row0 + r);
+                if (r + 64 <= npad) {
+                    tma_load_2d(dst + r * 128, &tx64, &full[s], kc, row0 + r);
+                    r += 64;
+                }
+                if (r + 32 <= npad) {
+                    tma_load_2d(dst + r * 128, &tx32, &full[s], kc, row0 + r);
+                    r += 32;
+                }
+                if (r + 16 <= npad) tma_load_2d(dst + r * 128, &tx16, &full[s], kc, row0 + r);
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
+    } else if (warp == 1 || warp == PF_MMA2_WARP) {
+        // MMA issue for matrix m (GEMM1: warp 1 gate, warp 14 up; GEMM2: warp 1)
+        const int m = warp == 1 ? 0 : 1;
+        if (lane == 0 && m < C::NISSUE) {
             const uint32_t idesc = make_idesc_bf16(PF_BM, npad);
+            uint64_t* mdeq = deq + m * C::ASLOTS;
+            uint64_t* maempty = aempty + m * C::ASLOTS;
             for (int mt = 0; mt < nmt && alive; ++mt) {
                 const int buf = mt % C::NACC, use = mt / C::NACC;
-                if (!mbar_wait(&acce[buf], (use & 1) ^ 1)) { alive = false; break; }  // drained by the epilogue
+                if (!mbar_wait_fast(&acce[buf], (use & 1) ^ 1)) { alive = false; break; }  // drained by the epilogue
                 tc_fence_after();
-                const uint32_t dcol = tmem + buf * C::ACC_COLS;
-                for (int kb = 0; kb < nk; ++kb) {
+                const uint32_t dcol = tmem + buf * C::ACC_COLS + m * C::MAT_COLS;
+                for (int kb = 0; kb < nk && alive; ++kb) {
                     const int i = mt * nk + kb;
                     const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-                    const int sa = i % C::ASTAGES, pa = (i / C::ASTAGES) & 1;
-                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&deq[sa], pa)) { alive = false; break; }
-                    tc_fence_after();
+                    if (!mbar_wait_fast(&full[s], ph)) { alive = false; break; }
                     const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
-                        const uint64_t bdesc = make_sdesc_sw128(bb + kk * 32);
+                    for (int kh = 0; kh < 2; ++kh) {
+                        const int j = 2 * i + kh, sl = j % C::ASLOTS;
+                        if (!mbar_wait_fast(&mdeq[sl], (j / C::ASLOTS) & 1)) { alive = false; break; }
+                        tc_fence_after();
+                        const uint32_t acol = tmem + C::A_COL0 + sl * C::SLOT_COLS + m * (PF_AK / 2);
 #pragma unroll
-                        for (int m = 0; m < C::NMAT; ++m) {
-                            const uint32_t ab = smem_u32(sA + (sa * C::NMAT + m) * C::A_BYTES);
-                            tc_mma_bf16(dcol + m * C::MAT_COLS, make_sdesc_sw128(ab + kk * 32), bdesc, idesc,
-                                        (kb | kk) != 0);
-                        }
+                        for (int k2 = 0; k2 < 2; ++k2)
+                            tc_mma_bf16_ts(dcol, acol + k2 * 8, make_sdesc_sw128(bb + (2 * kh + k2) * 32), idesc,
+                                           (kb | kh | k2) != 0);
+                        tc_commit(&maempty[sl]);  // the A slot may be rewritten
                     }
-                    tc_commit(&empty[s]);    // the activation tile may be refilled
-                    tc_commit(&aempty[sa]);  // the A tile may be rewritten
+                    tc_commit(&empty[s]);  // this matrix is done with the activation tile
                 }
                 tc_commit(&accf[buf]);
             }
         }
-    } else if (warp >= PF_DQ_WARP0) {
-        const int dt = threadIdx.x - PF_DQ_WARP0 * 32;  // 0..255
-        const int row = dt >> 1, half = dt & 1;
+    } else if (warp >= PF_DQ_WARP0 && warp < PF_DQ_WARP0 + PF_DQ_THREADS / 32) {
+        // Warp (quadrant q, group g) owns weight rows 32 q .. 32 q + 31 of the
+        // M-tile, one row per lane (its TMEM lane), and one 32-element block of
+        // them per stage it takes.  GEMM1: group g = (matrix g / 2, half g % 2)
+        // of every stage.  GEMM2: half g % 2 of every other stage (parity g / 2).
+        const int q = warp & 3, grp = (warp - PF_DQ_WARP0) >> 2;
+        const int m = MODE == 0 ? grp >> 1 : 0;       // matrix
+        const int half = grp & 1;                     // block of the stage
+        const int i0 = MODE == 0 ? 0 : grp >> 1;      // first stage taken
+        constexpr int STRIDE = MODE == 0 ? 1 : 2;     // stages between the ones taken
+        uint64_t* mdeq = deq + m * C::ASLOTS;
+        uint64_t* maempty = aempty + m * C::ASLOTS;
+        const int row = q * 32 + lane;
         const uint8_t* sbase = a.arena + slot * a.slot_bytes;
-        const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[MODE == 0 ? 0 : 2]);
-        const uint16_t* sc1 = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[1]);
-        // One 16-byte load holds this thread's scales for 4 consecutive stages (blocks
-        // 2 kb .. 2 kb + 7 of its row); when nk % 4 == 0 groups of 4 stages never
-        // straddle an M-tile and the next group's scales are loaded a group ahead.
-        // Otherwise (K % 256 != 0) each stage loads its own scale.
-        const bool grouped = (nk & 3) == 0;
-        const int ngrp = grouped ? nstage / 4 : 0;
-        auto load_grp = [&](int gi, uint4& r0, uint4& r1) {
-            const int i0 = gi * 4, kb0 = i0 % nk;
-            const size_t base = (size_t)((mt0 + i0 / nk) * PF_BM + row) * (K / 32) + 2 * kb0;
-            r0 = __ldg(reinterpret_cast<const uint4*>(sc0 + base));
-            if (C::NMAT == 2) r1 = __ldg(reinterpret_cast<const uint4*>(sc1 + base));
+        const int mi = MODE == 0 ? m : 2;             // arena matrix index
+        const uint8_t* cb = sbase + a.off_codes[mi];
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[mi]);
+        const int bits = MODE == 0 ? (m == 0 ? B0 : B1) : B0;
+        const int nb = K / 32;  // blocks (and scales) per weight row
+        const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + C::A_COL0 + m * (PF_AK / 2);
+        const int ntake = nstage > i0 ? (nstage - i0 + STRIDE - 1) / STRIDE : 0;  // stages this warp takes
+        struct Pre {
+            uint4 c;
+            float s;
         };
-        auto pick = [](const uint4& v, int idx) -> uint16_t {  // half idx (0..7) of v
-            const int wi = idx >> 1;
-            const uint32_t w = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
-            return (uint16_t)(w >> (16 * (idx & 1)));
+        auto fetch = [&](int t, Pre& p) {  // t-th stage taken
+            if (t >= ntake) return;
+            const int i = i0 + t * STRIDE, mt = i / nk;
+            const size_t blk = ((size_t)(mt0 + mt) * PF_BM + row) * nb + 2 * (i - mt * nk) + half;
+            p.c = bits == 4 ? load_block_codes<4>(cb + blk * 16) : load_block_codes<2>(cb + blk * 8);
+            p.s = half_bits_to_f32(__ldg(sc + blk));
         };
-        uint4 cur0 = make_uint4(0, 0, 0, 0), cur1 = cur0, nxt0 = cur0, nxt1 = cur0;
-        if (ngrp > 0) load_grp(0, cur0, cur1);
-        if (ngrp > 1) load_grp(1, nxt0, nxt1);
-        for (int i = 0; i < nstage; ++i) {
-            const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-            const int sa = i % C::ASTAGES, pa = (i / C::ASTAGES) & 1;
-            uint16_t q0, q1 = 0;
-            if (grouped) {
-                if ((i & 3) == 0 && i > 0) {
-                    cur0 = nxt0;
-                    cur1 = nxt1;
-                    if ((i >> 2) + 1 < ngrp) load_grp((i >> 2) + 1, nxt0, nxt1);
-                }
-                const int si = 2 * (i & 3) + half;
-                q0 = pick(cur0, si);
-                if (C::NMAT == 2) q1 = pick(cur1, si);
-            } else {
-                const size_t grow = (size_t)((mt0 + i / nk) * PF_BM + row);  // weight row in the matrix
-                q0 = __ldg(sc0 + grow * (K / 32) + 2 * (i % nk) + half);
-                if (C::NMAT == 2) q1 = __ldg(sc1 + grow * (K / 32) + 2 * (i % nk) + half);
-            }
-            if (!mbar_wait(&full[s], ph) || !mbar_wait(&aempty[sa], pa ^ 1)) { alive = false; break; }
-            dequant_unit<B0>(sC + (s * C::NMAT + 0) * C::C_BYTES, sA + (sa * C::NMAT + 0) * C::A_BYTES, row, half,
-                             half_bits_to_f32(q0));
-            if (C::NMAT == 2)
-                dequant_unit<B1>(sC + (s * C::NMAT + 1) * C::C_BYTES, sA + (sa * C::NMAT + 1) * C::A_BYTES, row,
-                                 half, half_bits_to_f32(q1));
-            fence_proxy_async_smem();
+        auto step = [&](int t, const Pre& p) -> bool {
+            const int j = 2 * (i0 + t * STRIDE) + half, sl = j % C::ASLOTS;
+            if (!mbar_wait_fast(&maempty[sl], ((j / C::ASLOTS) & 1) ^ 1)) return false;
+            tc_fence_after();
+            uint32_t col[16];
+            if (bits == 4) dequant_block_cols<4>(p.c, p.s, col);
+            else dequant_block_cols<2>(p.c, p.s, col);
+            tmem_st16(tcol + sl * C::SLOT_COLS, col);
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&deq[sa]);
-                mbar_arrive(&empty[s]);  // this warp's reads of the codes are done
-            }
+            if (lane == 0) mbar_arrive(&mdeq[sl]);
+            return true;
+        };
+        static_assert(PF_PREFETCH == 4, "the loop below holds four stages in p0..p3");
+        Pre p0{}, p1{}, p2{}, p3{};
+        fetch(0, p0);
+        fetch(1, p1);
+        fetch(2, p2);
+        fetch(3, p3);
+        for (int t = 0; t < ntake; t += 4) {
+            if (!step(t, p0)) break;
+            fetch(t + 4, p0);
+            if (t + 1 >= ntake || !step(t + 1, p1)) break;
+            fetch(t + 5, p1);
+            if (t + 2 >= ntake || !step(t + 2, p2)) break;
+            fetch(t + 6, p2);
+            if (t + 3 >= ntake || !step(t + 3, p3)) break;
+            fetch(t + 7, p3);
         }
-    } else {  // epilogue warps: TMEM -> registers -> global, one M-tile at a time
-        const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    } else if (warp >= PF_EPI_WARP0 && warp < PF_EPI_WARP0 + 4) {
+        // epilogue warps: TMEM -> registers -> global, one M-tile at a time.
+        // Lane l of warp q holds output feature 32 q + l of the M-tile for 16
+        // consecutive pair rows at a time (the next 16 are loaded meanwhile).
+        // Neighbouring lanes swap values so that each stores a bf16 pair:
+        // the even lane features (l, l + 1) of row j, the odd lane features
+        // (l - 1, l) of row j + 1.
+        const int q = warp & 3;
+        const int odd = lane & 1;
         for (int mt = 0; mt < nmt && alive; ++mt) {
             const int buf = mt % C::NACC, use = mt / C::NACC;
-            if (!mbar_wait(&accf[buf], use & 1)) { alive = false; break; }
+            if (!mbar_wait_fast(&accf[buf], use & 1)) { alive = false; break; }
             tc_fence_after();
-            const int r = (mt0 + mt) * PF_BM + q * 32 + lane;  // output feature of this thread
+            const int f = (mt0 + mt) * PF_BM + q * 32 + (lane & ~1);  // first feature of this lane's pair
             const uint32_t ta0 = tmem + buf * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
+            uint32_t g[16], u[16];
+            tmem_ld16(ta0, g);
+            if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS, u);
             for (int c0 = 0; c0 < npad; c0 += 16) {
-                uint32_t v0[16], v1[16];
-                tmem_ld16(ta0 + c0, v0);
-                if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0, v1);
-                tmem_ld_wait();
+                tmem_ld_wait16(g);
+                if (MODE == 0) reg_tie16(u);
+                float o[16];
+                if (MODE == 0) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = c0 + j;
-                    if (n < nrows) {
-                        float o;
-                        if (MODE == 0) o = silu_f32(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
-                        else o = s_w[n] * __uint_as_float(v0[j]);
-                        a.out[(size_t)(row0 + n) * NOUT + r] = f32_to_bf16_bits(o);
+                    for (int j = 0; j < 16; ++j) {
+                        const float x = __uint_as_float(g[j]);
+                        o[j] = __fdividef(x, 1.0f + __expf(-x)) * __uint_as_float(u[j]);
                     }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(s_w + c0 + j);  // rows past nrows: unused
+                        o[j] = w4.x * __uint_as_float(g[j]);
+                        o[j + 1] = w4.y * __uint_as_float(g[j + 1]);
+                        o[j + 2] = w4.z * __uint_as_float(g[j + 2]);
+                        o[j + 3] = w4.w * __uint_as_float(g[j + 3]);
+                    }
+                }
+                if (c0 + 16 < npad) {  // the next 16 columns load while these are stored
+                    tmem_ld16(ta0 + c0 + 16, g);
+                    if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0 + 16, u);
+                }
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[j] : o[j + 1], 1);
+                    const uint32_t pk = odd ? pack_bf16x2(recv, o[j + 1]) : pack_bf16x2(o[j], recv);
+                    const int n = c0 + j + odd;
+                    if (n < nrows) *reinterpret_cast<uint32_t*>(a.out + (size_t)(row0 + n) * NOUT + f) = pk;
                 }
             }
             tc_fence_before();

@@ -16,7 +16,7 @@
 // shared memory holds only the activation tiles and the tensor core reads
 // only B from it.  TMEM (512 columns): the accumulators (gate and up for
 // GEMM1, two buffers for GEMM2, PF_BN_MAX columns each) and, above them, a
-// ring of A slots, each K = 32 of every weight matrix (16 columns per matrix).
+// ring of A slots, each one stage (K = 64, 32 columns) of every weight matrix.
 //
 // A CTA owns one N-tile and walks its M-tiles, so the activation rows stay in
 // L2 and setup is paid once.  Roles (448 threads): warp 0 issues the TMA loads
@@ -35,7 +35,6 @@
 #include "common.cuh"
 
 #define PF_BK 64          // K elements per stage (one 128-byte swizzle row of bf16)
-#define PF_AK 32          // K elements per A slot (one quantisation block)
 #define PF_BM 128         // weight rows per M-tile
 #define PF_BN_MAX 192     // pair rows per tile (PREFILL_TILE_N)
 #define PF_EPI_WARP0 2    // epilogue warps 2..5 (TMEM lane quadrants 2, 3, 0, 1)
@@ -53,16 +52,16 @@ struct PfCfg {
     static constexpr int MAT_COLS = PF_BN_MAX;                   // TMEM columns of one matrix's accumulator
     static constexpr int ACC_COLS = NMAT * PF_BN_MAX;            // TMEM columns of one accumulator buffer
     static constexpr int A_COL0 = NACC * ACC_COLS;               // first TMEM column of the A slots
-    static constexpr int SLOT_COLS = NMAT * (PF_AK / 2);         // TMEM columns of one A slot
+    static constexpr int SLOT_COLS = NMAT * (PF_BK / 2);         // TMEM columns of one A slot (one stage)
     static constexpr int TMEM_COLS = 512;
-    static constexpr int ASLOTS = (TMEM_COLS - A_COL0) / SLOT_COLS;  // 4 (GEMM1) or 8 (GEMM2)
+    static constexpr int ASLOTS = (TMEM_COLS - A_COL0) / SLOT_COLS;  // 2 (GEMM1) or 4 (GEMM2)
     static constexpr int NISSUE = NMAT;                          // MMA-issuing threads, one per matrix
-    // A-slot arrivals per matrix: the four dequant warps (one per TMEM lane quadrant) writing it
-    static constexpr int DQ_ARRIVALS = 4;
+    // arrivals on a matrix's A slot: one dequant warp per (TMEM lane quadrant, half of the stage)
+    static constexpr int DQ_ARRIVALS = 8;
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
-    static_assert(A_COL0 + ASLOTS * SLOT_COLS <= TMEM_COLS && ASLOTS >= 4, "TMEM budget");
+    static_assert(A_COL0 + ASLOTS * SLOT_COLS <= TMEM_COLS && ASLOTS >= 2, "TMEM budget");
     static_assert((2 * TSTAGES + 2 * NMAT * ASLOTS + 2 * NACC) * 8 + 4 <= BAR_BYTES, "barrier area");
 };
 
@@ -152,8 +151,7 @@ __device__ __forceinline__ void dequant_block_cols(uint4 c, float s, uint32_t (&
 
 // One CTA per (N-tile, M-tile group): expert e, rows row0 .. row0+nrows of the
 // grouped activations, M-tiles mt0 .. mt0+nmt of the output features.  Stage i
-// covers (M-tile mt0 + i / nk, K-block i % nk) and A slots 2i, 2i + 1 (its two
-// halves).  The four tensor maps view the same activation matrix with boxes of
+// covers (M-tile mt0 + i / nk, K-block i % nk) and A slot i % ASLOTS.  The four tensor maps view the same activation matrix with boxes of
 // 128, 64, 32 and 16 rows.
 template <int MODE, int B0, int B1>
 __global__ void __launch_bounds__(PF_THREADS, 1)
@@ -248,7 +246,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             }
         }
     } else if (warp == 1 || warp == PF_MMA2_WARP) {
-        // MMA issue for matrix m (GEMM1: warp 1 gate, warp 14 up; GEMM2: warp 1)
+        // MMA issue for matrix m (GEMM1: warp 1 gate, warp 22 up; GEMM2: warp 1)
         const int m = warp == 1 ? 0 : 1;
         if (lane == 0 && m < C::NISSUE) {
             const uint32_t idesc = make_idesc_bf16(PF_BM, npad);
@@ -262,21 +260,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 for (int kb = 0; kb < nk && alive; ++kb) {
                     const int i = mt * nk + kb;
                     const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-                    if (!mbar_wait_fast(&full[s], ph)) { alive = false; break; }
-                    const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
-#pragma unroll
-                    for (int kh = 0; kh < 2; ++kh) {
-                        const int j = 2 * i + kh, sl = j % C::ASLOTS;
-                        if (!mbar_wait_fast(&mdeq[sl], (j / C::ASLOTS) & 1)) { alive = false; break; }
-                        tc_fence_after();
-                        const uint32_t acol = tmem + C::A_COL0 + sl * C::SLOT_COLS + m * (PF_AK / 2);
-#pragma unroll
-                        for (int k2 = 0; k2 < 2; ++k2)
-                            tc_mma_bf16_ts(dcol, acol + k2 * 8, make_sdesc_sw128(bb + (2 * kh + k2) * 32), idesc,
-                                           (kb | kh | k2) != 0);
-                        tc_commit(&maempty[sl]);  // the A slot may be rewritten
+                    const int sl = i % C::ASLOTS;
+                    if (!mbar_wait_fast(&full[s], ph) || !mbar_wait_fast(&mdeq[sl], (i / C::ASLOTS) & 1)) {
+                        alive = false;
+                        break;
                     }
-                    tc_commit(&empty[s]);  // this matrix is done with the activation tile
+                    tc_fence_after();
+                    const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
+                    const uint32_t acol = tmem + C::A_COL0 + sl * C::SLOT_COLS + m * (PF_BK / 2);
+#pragma unroll
+                    for (int kk = 0; kk < PF_BK / 16; ++kk)
+                        tc_mma_bf16_ts(dcol, acol + kk * 8, make_sdesc_sw128(bb + kk * 32), idesc, (kb | kk) != 0);
+                    tc_commit(&maempty[sl]);  // the A slot may be rewritten
+                    tc_commit(&empty[s]);     // this matrix is done with the activation tile
                 }
                 tc_commit(&accf[buf]);
             }
@@ -300,7 +296,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(sbase + a.off_scales[mi]);
         const int bits = MODE == 0 ? (m == 0 ? B0 : B1) : B0;
         const int nb = K / 32;  // blocks (and scales) per weight row
-        const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + C::A_COL0 + m * (PF_AK / 2);
+        const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + C::A_COL0 + m * (PF_BK / 2) + half * 16;
         const int ntake = nstage > i0 ? (nstage - i0 + STRIDE - 1) / STRIDE : 0;  // stages this warp takes
         struct Pre {
             uint4 c;
@@ -314,8 +310,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             p.s = half_bits_to_f32(__ldg(sc + blk));
         };
         auto step = [&](int t, const Pre& p) -> bool {
-            const int j = 2 * (i0 + t * STRIDE) + half, sl = j % C::ASLOTS;
-            if (!mbar_wait_fast(&maempty[sl], ((j / C::ASLOTS) & 1) ^ 1)) return false;
+            const int i = i0 + t * STRIDE, sl = i % C::ASLOTS;
+            if (!mbar_wait_fast(&maempty[sl], ((i / C::ASLOTS) & 1) ^ 1)) return false;
             tc_fence_after();
             uint32_t col[16];
             if (bits == 4) dequant_block_cols<4>(p.c, p.s, col);

@@ -63,6 +63,7 @@ struct PfCfg {
     static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
     static_assert(A_COL0 + ASLOTS * SLOT_COLS <= TMEM_COLS && ASLOTS >= 2, "TMEM budget");
     static_assert((2 * TSTAGES + 2 * NMAT * ASLOTS + 2 * NACC) * 8 + 4 <= BAR_BYTES, "barrier area");
+    static_assert(PF_BK == 64 && TSTAGES * B_BYTES + 2048 < (1 << 18), "B descriptors as offsets of one base");
 };
 
 struct PrefillArgs {
@@ -226,9 +227,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             tma_prefetch_desc(&tx32);
             tma_prefetch_desc(&tx16);
             const uint32_t bytes = npad * PF_BK * 2;
+            int s = 0, ph = 0, kb = 0;
             for (int i = 0; i < nstage; ++i) {
-                const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-                const int kc = (i % nk) * PF_BK;
+                const int kc = kb * PF_BK;
                 if (!mbar_wait_fast(&empty[s], ph ^ 1)) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 uint8_t* dst = sB + s * C::B_BYTES;  // row r at r * 128 B
@@ -243,36 +244,46 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     r += 32;
                 }
                 if (r + 16 <= npad) tma_load_2d(dst + r * 128, &tx16, &full[s], kc, row0 + r);
+                if (++s == C::TSTAGES) { s = 0; ph ^= 1; }
+                if (++kb == nk) kb = 0;
             }
         }
     } else if (warp == 1 || warp == PF_MMA2_WARP) {
         // MMA issue for matrix m (GEMM1: warp 1 gate, warp 22 up; GEMM2: warp 1)
         const int m = warp == 1 ? 0 : 1;
         if (lane == 0 && m < C::NISSUE) {
+            // The issuing thread shares its SM sub-partition with four busy
+            // dequant warps, so its loop is kept short: ring positions advance
+            // incrementally and the B descriptors are offsets of one base (the
+            // whole ring lies below 256 KB, inside the descriptor's 14-bit
+            // address field, so the additions cannot carry out of it).
             const uint32_t idesc = make_idesc_bf16(PF_BM, npad);
             uint64_t* mdeq = deq + m * C::ASLOTS;
             uint64_t* maempty = aempty + m * C::ASLOTS;
+            const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(sB));
+            const uint32_t abase = tmem + C::A_COL0 + m * (PF_BK / 2);
+            int s = 0, ph = 0, sl = 0, pa = 0;
             for (int mt = 0; mt < nmt && alive; ++mt) {
                 const int buf = mt % C::NACC, use = mt / C::NACC;
                 if (!mbar_wait_fast(&acce[buf], (use & 1) ^ 1)) { alive = false; break; }  // drained by the epilogue
                 tc_fence_after();
                 const uint32_t dcol = tmem + buf * C::ACC_COLS + m * C::MAT_COLS;
-                for (int kb = 0; kb < nk && alive; ++kb) {
-                    const int i = mt * nk + kb;
-                    const int s = i % C::TSTAGES, ph = (i / C::TSTAGES) & 1;
-                    const int sl = i % C::ASLOTS;
-                    if (!mbar_wait_fast(&full[s], ph) || !mbar_wait_fast(&mdeq[sl], (i / C::ASLOTS) & 1)) {
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_fast(&full[s], ph) || !mbar_wait_fast(&mdeq[sl], pa)) {
                         alive = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
-                    const uint32_t acol = tmem + C::A_COL0 + sl * C::SLOT_COLS + m * (PF_BK / 2);
-#pragma unroll
-                    for (int kk = 0; kk < PF_BK / 16; ++kk)
-                        tc_mma_bf16_ts(dcol, acol + kk * 8, make_sdesc_sw128(bb + kk * 32), idesc, (kb | kk) != 0);
+                    const uint64_t bd = bdesc0 + (uint32_t)(s * (C::B_BYTES >> 4));
+                    const uint32_t ac = abase + sl * C::SLOT_COLS;
+                    tc_mma_bf16_ts(dcol, ac, bd, idesc, kb != 0);
+                    tc_mma_bf16_ts(dcol, ac + 8, bd + 2, idesc, 1u);   // K 16..31: +32 bytes
+                    tc_mma_bf16_ts(dcol, ac + 16, bd + 4, idesc, 1u);
+                    tc_mma_bf16_ts(dcol, ac + 24, bd + 6, idesc, 1u);
                     tc_commit(&maempty[sl]);  // the A slot may be rewritten
                     tc_commit(&empty[s]);     // this matrix is done with the activation tile
+                    if (++s == C::TSTAGES) { s = 0; ph ^= 1; }
+                    if (++sl == C::ASLOTS) { sl = 0; pa ^= 1; }
                 }
                 tc_commit(&accf[buf]);
             }

@@ -428,12 +428,28 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         if (lane == 0) a.slow_list[atomicAdd(a.slow_count, 1)] = t;
         return;
     }
-    // 3) prefill: re-evaluate the candidates in fp64 (all at once, lane-strided)
+    // 3) prefill: re-evaluate in fp64 (lane-strided) the candidates that the
+    //    certification could not separate: both ends of every overlapping
+    //    adjacent pair among the k + 1 best (the lanes are in rank order after
+    //    sort_and_certify).  The others keep their fast values and bounds,
+    //    which still contain the exact logits, so the second certification
+    //    below is as valid as the first.
     if (MODE == 0) {
-        for (int base = 0; base < MC; base += 16) {
-            int ej[16];
+        const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
+        const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
+        const bool pairbad = lane < k && lane + 1 < MC && !((cval - cbnd) > (nv + nb));
+        const bool prevbad = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0 && lane > 0;
+        const unsigned need = __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad));
+        const int NR = __popc(need);
+        for (int base = 0; base < NR; base += 16) {
+            int ej[16], lj[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) ej[j] = __shfl_sync(0xffffffffu, ce, min(base + j, 31));
+            for (int j = 0; j < 16; ++j) {  // lane of the (base + j)-th flagged candidate
+                unsigned mm = need;
+                for (int z = 0; z < base + j && mm; ++z) mm &= mm - 1;
+                lj[j] = mm ? __ffs(mm) - 1 : 31;
+                ej[j] = __shfl_sync(0xffffffffu, ce, lj[j]);
+            }
             double acc[16], ab[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = ab[j] = 0.0;
@@ -443,7 +459,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
                 const double xd = bf16_bits_to_f32(xr[h]);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (base + j < MC) {
+                    if (base + j < NR) {
                         const double p = xd * (double)__ldg(a.W + (size_t)ej[j] * H + h);
                         acc[j] += p;
                         ab[j] += fabs(p);
@@ -451,10 +467,10 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                if (base + j < MC) {
+                if (base + j < NR) {
                     const double s = warp_sum_d(acc[j]), sa = warp_sum_d(ab[j]);
                     const double bb = a.b ? (double)a.b[ej[j]] : 0.0;
-                    if (lane == base + j) {
+                    if (lane == lj[j]) {
                         cval = s + bb;
                         cbnd = (sa + fabs(bb)) * (1.0 + 1e-9) * (g_par + g_or) + 1e-300;
                     }

@@ -71,16 +71,21 @@ __global__ void __launch_bounds__(MOE_MAX_E) k_perm_scan(PermArgs a) {
     const int e = threadIdx.x;
     int c = 0;
     if (e < a.E)
-        for (int b = 0; b < a.nchunks; ++b) {
-            int v = a.chunk_cnt[(size_t)b * a.E + e];
-            a.chunk_cnt[(size_t)b * a.E + e] = c;  // relative base of chunk b
-            c += v;
+        for (int b0 = 0; b0 < a.nchunks; b0 += 16) {  // 16 loads in flight, then their bases
+            int v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = b0 + j < a.nchunks ? a.chunk_cnt[(size_t)(b0 + j) * a.E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (b0 + j < a.nchunks) {
+                    a.chunk_cnt[(size_t)(b0 + j) * a.E + e] = c;  // relative base of chunk b0 + j
+                    c += v[j];
+                }
         }
     int off;
     int total = block_excl_scan(c, &off, s_warp);
     if (e < a.E) {
-        a.offsets[e] = off;
-        for (int b = 0; b < a.nchunks; ++b) a.chunk_cnt[(size_t)b * a.E + e] += off;
+        a.offsets[e] = off;  // chunk b of expert e starts at offsets[e] + chunk_cnt[b][e]
         if (a.hist) a.hist[(size_t)a.layer * a.E + e] += (uint32_t)c;
     }
     if (e == 0) a.offsets[a.E] = total;
@@ -106,7 +111,8 @@ __global__ void __launch_bounds__(MOE_MAX_E) k_perm_scan(PermArgs a) {
 
 __global__ void __launch_bounds__(PERM_CHUNK) k_perm_scatter(PermArgs a) {
     __shared__ int cursor[MOE_MAX_E];
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) cursor[e] = a.chunk_cnt[(size_t)blockIdx.x * a.E + e];
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+        cursor[e] = a.offsets[e] + a.chunk_cnt[(size_t)blockIdx.x * a.E + e];
     __syncthreads();
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int p = blockIdx.x * PERM_CHUNK + threadIdx.x;

@@ -58,6 +58,11 @@ struct PfCfg {
     static constexpr int NISSUE = NMAT;                          // MMA-issuing threads, one per matrix
     // arrivals on a matrix's A slot: one dequant warp per (TMEM lane quadrant, half of the stage)
     static constexpr int DQ_ARRIVALS = 8;
+    // The 4 epilogue warps drain the accumulators.  (Letting the dequant warps
+    // take part in GEMM1's drain, which stalls its MMAs, made GEMM1 slower:
+    // the drain's registers spill in the dequant loop.)
+    static constexpr int DRAIN_PARTS = 1;
+    static constexpr int DRAIN_ARRIVALS = 4;
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&accf[b], C::NISSUE);
-            mbar_init(&acce[b], 4);
+            mbar_init(&acce[b], C::DRAIN_ARRIVALS);
         }
         fence_mbar_init();
     }
@@ -219,6 +224,65 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool alive = true;
+
+    // Drains M-tile mt's accumulator from this warp's TMEM lane quadrant:
+    // chunks part, part + nparts, ... of 16 columns (the next chunk loads while
+    // one is stored), then one arrival on the accumulator's "drained" barrier.
+    // Lane l holds output feature 32 q + l of the M-tile; neighbouring lanes
+    // swap values so that each stores a bf16 pair: the even lane features
+    // (l, l + 1) of row j, the odd lane features (l - 1, l) of row j + 1.
+    auto drain = [&](int mt, int part, int nparts) -> bool {
+        const int q = warp & 3, odd = lane & 1;
+        const int buf = mt % C::NACC, use = mt / C::NACC;
+        if (!mbar_wait_fast(&accf[buf], use & 1)) return false;
+        __syncwarp();  // converged for the .aligned TMEM loads
+        tc_fence_after();
+        const int f = (mt0 + mt) * PF_BM + q * 32 + (lane & ~1);  // first feature of this lane's pair
+        const uint32_t ta0 = tmem + buf * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
+        const int step = 16 * nparts;
+        uint32_t g[16], u[16];
+        int c0 = 16 * part;
+        if (c0 < npad) {
+            tmem_ld16(ta0 + c0, g);
+            if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0, u);
+        }
+        for (; c0 < npad; c0 += step) {
+            tmem_ld_wait16(g);
+            if (MODE == 0) reg_tie16(u);
+            float o[16];
+            if (MODE == 0) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float x = __uint_as_float(g[j]);
+                    o[j] = __fdividef(x, 1.0f + __expf(-x)) * __uint_as_float(u[j]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(s_w + c0 + j);  // rows past nrows: unused
+                    o[j] = w4.x * __uint_as_float(g[j]);
+                    o[j + 1] = w4.y * __uint_as_float(g[j + 1]);
+                    o[j + 2] = w4.z * __uint_as_float(g[j + 2]);
+                    o[j + 3] = w4.w * __uint_as_float(g[j + 3]);
+                }
+            }
+            if (c0 + step < npad) {  // the next chunk loads while this one is stored
+                tmem_ld16(ta0 + c0 + step, g);
+                if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0 + step, u);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[j] : o[j + 1], 1);
+                const uint32_t pk = odd ? pack_bf16x2(recv, o[j + 1]) : pack_bf16x2(o[j], recv);
+                const int n = c0 + j + odd;
+                if (n < nrows) *reinterpret_cast<uint32_t*>(a.out + (size_t)(row0 + n) * NOUT + f) = pk;
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[buf]);
+        return true;
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -351,59 +415,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             fetch(t + 7, p3);
         }
     } else if (warp >= PF_EPI_WARP0 && warp < PF_EPI_WARP0 + 4) {
-        // epilogue warps: TMEM -> registers -> global, one M-tile at a time.
-        // Lane l of warp q holds output feature 32 q + l of the M-tile for 16
-        // consecutive pair rows at a time (the next 16 are loaded meanwhile).
-        // Neighbouring lanes swap values so that each stores a bf16 pair:
-        // the even lane features (l, l + 1) of row j, the odd lane features
-        // (l - 1, l) of row j + 1.
-        const int q = warp & 3;
-        const int odd = lane & 1;
-        for (int mt = 0; mt < nmt && alive; ++mt) {
-            const int buf = mt % C::NACC, use = mt / C::NACC;
-            if (!mbar_wait_fast(&accf[buf], use & 1)) { alive = false; break; }
-            tc_fence_after();
-            const int f = (mt0 + mt) * PF_BM + q * 32 + (lane & ~1);  // first feature of this lane's pair
-            const uint32_t ta0 = tmem + buf * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
-            uint32_t g[16], u[16];
-            tmem_ld16(ta0, g);
-            if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS, u);
-            for (int c0 = 0; c0 < npad; c0 += 16) {
-                tmem_ld_wait16(g);
-                if (MODE == 0) reg_tie16(u);
-                float o[16];
-                if (MODE == 0) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float x = __uint_as_float(g[j]);
-                        o[j] = __fdividef(x, 1.0f + __expf(-x)) * __uint_as_float(u[j]);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; j += 4) {
-                        const float4 w4 = *reinterpret_cast<const float4*>(s_w + c0 + j);  // rows past nrows: unused
-                        o[j] = w4.x * __uint_as_float(g[j]);
-                        o[j + 1] = w4.y * __uint_as_float(g[j + 1]);
-                        o[j + 2] = w4.z * __uint_as_float(g[j + 2]);
-                        o[j + 3] = w4.w * __uint_as_float(g[j + 3]);
-                    }
-                }
-                if (c0 + 16 < npad) {  // the next 16 columns load while these are stored
-                    tmem_ld16(ta0 + c0 + 16, g);
-                    if (MODE == 0) tmem_ld16(ta0 + C::MAT_COLS + c0 + 16, u);
-                }
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
-                    const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[j] : o[j + 1], 1);
-                    const uint32_t pk = odd ? pack_bf16x2(recv, o[j + 1]) : pack_bf16x2(o[j], recv);
-                    const int n = c0 + j + odd;
-                    if (n < nrows) *reinterpret_cast<uint32_t*>(a.out + (size_t)(row0 + n) * NOUT + f) = pk;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[buf]);
-        }
+        // epilogue warps: part 0 of every M-tile's drain
+        for (int mt = 0; mt < nmt && alive; ++mt) alive = drain(mt, 0, C::DRAIN_PARTS);
     }
     tc_fence_before();
     __syncthreads();

@@ -215,3 +215,49 @@ __global__ void k_combine(const uint16_t* __restrict__ x, const YT* __restrict__
     o.y = (uint32_t)f32_to_bf16_bits(acc[2]) | ((uint32_t)f32_to_bf16_bits(acc[3]) << 16);
     *reinterpret_cast<uint2*>(out + (size_t)t * H + c) = o;
 }
+
+
+// Prefill combine for bf16 Y: out[t][c..c+7] = sum_j Y[inv[t][j]][c..c+7] (+ x),
+// summed in j order in fp32; 16-byte loads, four rows in flight.
+__global__ void __launch_bounds__(128) k_combine_bf16x8(const uint16_t* __restrict__ x, const uint16_t* __restrict__ y,
+                                                        const int32_t* __restrict__ inv, int T, int H, int k,
+                                                        int residual, uint16_t* __restrict__ out) {
+    const int t = blockIdx.y;
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (t >= T || c >= H) return;
+    float acc[8];
+#pragma unroll
+    for (int z = 0; z < 8; ++z) acc[z] = 0.f;
+    const int32_t* iv = inv + (size_t)t * k;
+    for (int j0 = 0; j0 < k; j0 += 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j0 + j < k) v[j] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)__ldg(iv + j0 + j) * H + c));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j0 + j < k) {
+                const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    acc[2 * z] += __uint_as_float(w[z] << 16);
+                    acc[2 * z + 1] += __uint_as_float(w[z] & 0xffff0000u);
+                }
+            }
+    }
+    if (residual) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + c));
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+            acc[2 * z] += __uint_as_float(w[z] << 16);
+            acc[2 * z + 1] += __uint_as_float(w[z] & 0xffff0000u);
+        }
+    }
+    uint4 o;
+    o.x = (uint32_t)f32_to_bf16_bits(acc[0]) | ((uint32_t)f32_to_bf16_bits(acc[1]) << 16);
+    o.y = (uint32_t)f32_to_bf16_bits(acc[2]) | ((uint32_t)f32_to_bf16_bits(acc[3]) << 16);
+    o.z = (uint32_t)f32_to_bf16_bits(acc[4]) | ((uint32_t)f32_to_bf16_bits(acc[5]) << 16);
+    o.w = (uint32_t)f32_to_bf16_bits(acc[6]) | ((uint32_t)f32_to_bf16_bits(acc[7]) << 16);
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + c) = o;
+}

@@ -496,7 +496,7 @@ int run_prefill(const LayerCall& c) {
     uint16_t* xp = reinterpret_cast<uint16_t*>(c.ws + L.xp);
     uint16_t* h = reinterpret_cast<uint16_t*>(c.ws + L.h);
     uint16_t* y = reinterpret_cast<uint16_t*>(c.ws + L.y);
-    k_gather_rows<<<P, 128, 0, c.st>>>(c.x, r.perm, P, H, c.k, xp);
+    k_gather_rows<<<(P + GATHER_ROWS - 1) / GATHER_ROWS, 32 * GATHER_ROWS, 0, c.st>>>(c.x, r.perm, P, H, c.k, xp);
     ActMaps tx, th;
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
     if (!tx.make(xp, P, H) || !th.make(h, P, I)) return MOE_ERR_CUDA;
@@ -520,7 +520,7 @@ int run_prefill(const LayerCall& c) {
     if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, a, H / PF_BM, mg2, nt, c.st);
     else launch_gemm<1, 2, 2>(th, a, H / PF_BM, mg2, nt, c.st);
     stage(3, c.st);
-    k_combine<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+    k_combine_bf16x8<<<dim3((H / 8 + 127) / 128, c.T), 128, 0, c.st>>>(
         c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);
     stage(4, c.st);
     count(4);

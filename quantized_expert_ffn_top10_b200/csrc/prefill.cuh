@@ -423,13 +423,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-// Xp[pos][:] = x[perm[pos] / k][:]  (gathered activation rows, bf16)
-__global__ void k_gather_rows(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int P, int H, int k,
-                              uint16_t* __restrict__ xp) {
-    const int pos = blockIdx.x;
+// Xp[pos][:] = x[perm[pos] / k][:]  (gathered activation rows, bf16).  One warp
+// per row, 8 rows per block; a lane's 16-byte loads are all issued before its
+// stores.
+#define GATHER_ROWS 8
+__global__ void __launch_bounds__(32 * GATHER_ROWS) k_gather_rows(const uint16_t* __restrict__ x,
+                                                                  const int32_t* __restrict__ perm, int P, int H,
+                                                                  int k, uint16_t* __restrict__ xp) {
+    const int pos = blockIdx.x * GATHER_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (pos >= P) return;
     const int t = perm[pos] / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)pos * H);
-    for (int i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = __ldg(src + i);
+    const int n = H / 8;  // 16-byte chunks per row
+    for (int i0 = lane; i0 < n; i0 += 32 * 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + 32 * j < n) v[j] = __ldg(src + i0 + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + 32 * j < n) dst[i0 + 32 * j] = v[j];
+    }
 }
+

@@ -509,8 +509,10 @@ int run_prefill(const LayerCall& c) {
     a.perm = r.perm; a.topk_w = r.w;
     const int nt = max_tiles(P, c.E);
     a.out = h;
-    // CTAs per N-tile (measured best at H = 2048, I = 512: two each, GEMM1 over 2 M-tiles, GEMM2 over 8)
-    const int mg1 = std::max(1, I / PF_BM / 2), mg2 = std::max(1, H / PF_BM / 8);
+    // CTAs per N-tile: GEMM1 one per M-tile (the CTAs of a tile are adjacent, so they read its
+    // activation rows together and share them through L2), GEMM2 one per 8 M-tiles (measured
+    // best at H = 2048, I = 512)
+    const int mg1 = std::max(1, I / PF_BM), mg2 = std::max(1, H / PF_BM / 8);
     if (d->bits_gate == 4 && d->bits_up == 4) launch_gemm<0, 4, 4>(tx, a, I / PF_BM, mg1, nt, c.st);
     else if (d->bits_gate == 2 && d->bits_up == 2) launch_gemm<0, 2, 2>(tx, a, I / PF_BM, mg1, nt, c.st);
     else if (d->bits_gate == 2) launch_gemm<0, 2, 4>(tx, a, I / PF_BM, mg1, nt, c.st);

@@ -18,19 +18,25 @@
 // GEMM1, two buffers for GEMM2, PF_BN_MAX columns each) and, above them, a
 // ring of A slots, each one stage (K = 64, 32 columns) of every weight matrix.
 //
-// A CTA owns one N-tile and walks its M-tiles, so the activation rows stay in
-// L2 and setup is paid once.  Roles (448 threads): warp 0 issues the TMA loads
-// of the activation tile (128-B swizzled K-major; a tile of npad rows goes as
-// at most one box each of 128, 64, 32 and 16 rows, since the TMA engine's cost
-// grows with the number of boxes); warp 1 owns TMEM and one of its threads
-// issues tcgen05.mma (GEMM1: for the gate matrix, while a thread of warp 22
-// issues the up matrix's: one thread issues at most one MMA per ~100 cycles,
-// about 80 cycles of tensor work at N = 160); warps 2-5 drain finished accumulators (TMEM -> registers
-// -> global; the down GEMM double-buffers them so this
-// overlaps the next M-tile); warps 6-21 load their own codes and scales from
-// the arena, PF_PREFETCH stages ahead in registers, and dequantise them into
-// the A slots (one 32-element block of 32 rows per warp and stage).  Rings: full / empty (activation tiles) and dequantised / free
-// (A slots) mbarriers; every wait is bounded.
+// A CTA owns one N-tile and a group of its M-tiles (GEMM1: one, GEMM2: eight);
+// the CTAs of an N-tile are adjacent in launch order, so they run together and
+// share its activation rows through L2.  Roles (736 threads):
+//   warp 0      TMA loads of the activation tile (128-B swizzled K-major; a
+//               tile of npad rows goes as at most one box each of 128, 64, 32
+//               and 16 rows, since the TMA engine's cost grows with the
+//               number of boxes);
+//   warp 1      owns TMEM; one thread issues tcgen05.mma (GEMM1: for the gate
+//               matrix, while a thread of warp 22 issues the up matrix's: one
+//               thread issues at most one MMA per ~100 cycles, about 80 cycles
+//               of tensor work at N = 160);
+//   warps 2-5   drain finished accumulators (TMEM -> registers -> global; the
+//               down GEMM double-buffers them so this overlaps the next
+//               M-tile);
+//   warps 6-21  load their own codes and scales from the arena, PF_PREFETCH
+//               stages ahead in registers, and dequantise them into the A
+//               slots (one 32-element block of 32 rows per warp and stage).
+// Rings: full / empty (activation tiles), dequantised / free (A slots) and
+// final / drained (accumulators) mbarriers; every wait is bounded.
 #pragma once
 #include "common.cuh"
 

@@ -49,11 +49,11 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.chunk = put(nch * E * 4);
     w.tiles = put((size_t)max_tiles((int)P, E) * 16);
     w.nrechk = put(4);
+    w.gbar = put(small ? DF_BAR_WORDS * 4 : 0);  // fused decode: grid barrier (right after nrechk: one memset clears both)
     w.xp = put(P * H * 2);
     w.h = put(P * I * (small ? 4 : 2));  // decode keeps h and Y in fp32, prefill in bf16
     w.y = put(P * H * (small ? 4 : 2));
     w.rec = put(small ? (size_t)DF_NREP * T * E * 16 : 0);  // fused decode: replicated (logit, bound) records
-    w.gbar = put(small ? DF_BAR_WORDS * 4 : 0);              // fused decode: grid barrier
     w.wsplit = put(small ? 0 : (size_t)3 * E * H * 2);        // chunk router: W_r as three bf16 planes
     w.xn = put(small ? 0 : (size_t)T * 4);                     // chunk router: ||x_t|| per token
     w.slow = put(small ? 0 : (size_t)(T + 4) * 4);             // chunk top-k: [count, tokens...] left to the slow pass
@@ -409,8 +409,15 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
                        d->off_codes[1] - d->off_codes[0], ns, sb) ||
         !tmap_codes_d(&tm[1], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb))
         return MOE_ERR_CUDA;
-    if (cudaMemsetAsync(a.bar, 0, DF_BAR_WORDS * 4, c.st) != cudaSuccess || cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess)
+    // the grid barrier's words and the recheck counter start at zero: one memset when the
+    // counter is the workspace's own (it sits just before the barrier words), else two
+    int32_t* const ws_nr = reinterpret_cast<int32_t*>(c.ws + L.nrechk);
+    if (a.nrechk == ws_nr) {
+        if (cudaMemsetAsync(ws_nr, 0, (L.gbar - L.nrechk) + DF_BAR_WORDS * 4, c.st) != cudaSuccess) return MOE_ERR_CUDA;
+    } else if (cudaMemsetAsync(a.bar, 0, DF_BAR_WORDS * 4, c.st) != cudaSuccess ||
+               cudaMemsetAsync(a.nrechk, 0, 4, c.st) != cudaSuccess) {
         return MOE_ERR_CUDA;
+    }
     stage(0, c.st);
     const int grid = g_df_grid[dev];
     cudaError_t e;

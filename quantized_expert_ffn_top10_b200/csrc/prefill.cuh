@@ -64,11 +64,12 @@ struct PfCfg {
     static constexpr int NISSUE = NMAT;                          // MMA-issuing threads, one per matrix
     // arrivals on a matrix's A slot: one dequant warp per (TMEM lane quadrant, half of the stage)
     static constexpr int DQ_ARRIVALS = 8;
-    // The 4 epilogue warps drain the accumulators.  (Letting the dequant warps
-    // take part in GEMM1's drain, which stalls its MMAs, made GEMM1 slower:
-    // the drain's registers spill in the dequant loop.)
-    static constexpr int DRAIN_PARTS = 1;
-    static constexpr int DRAIN_ARRIVALS = 4;
+    // The 4 epilogue warps drain the accumulators.  When a GEMM1 CTA has a
+    // single M-tile, its drain is the CTA's tail and the 16 dequant warps, done
+    // by then, take part: 5 warps per TMEM lane quadrant.  (Joining drains
+    // in the middle of the dequant loop made GEMM1 slower: the drain's
+    // registers spilled there.)
+    static constexpr int SHARED_DRAIN_PARTS = 1 + PF_DQ_THREADS / 128;
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
@@ -204,6 +205,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         return;
     }
 
+    const bool shared_drain = MODE == 0 && nmt == 1;
+    const int drain_parts = shared_drain ? C::SHARED_DRAIN_PARTS : 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::TSTAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&accf[b], C::NISSUE);
-            mbar_init(&acce[b], C::DRAIN_ARRIVALS);
+            mbar_init(&acce[b], shared_drain ? 4 + PF_DQ_THREADS / 32 : 4);
         }
         fence_mbar_init();
     }
@@ -410,19 +413,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         fetch(1, p1);
         fetch(2, p2);
         fetch(3, p3);
+        bool ok = true;
         for (int t = 0; t < ntake; t += 4) {
-            if (!step(t, p0)) break;
+            if (!(ok = step(t, p0))) break;
             fetch(t + 4, p0);
-            if (t + 1 >= ntake || !step(t + 1, p1)) break;
+            if (t + 1 >= ntake || !(ok = step(t + 1, p1))) break;
             fetch(t + 5, p1);
-            if (t + 2 >= ntake || !step(t + 2, p2)) break;
+            if (t + 2 >= ntake || !(ok = step(t + 2, p2))) break;
             fetch(t + 6, p2);
-            if (t + 3 >= ntake || !step(t + 3, p3)) break;
+            if (t + 3 >= ntake || !(ok = step(t + 3, p3))) break;
             fetch(t + 7, p3);
         }
+        if (shared_drain && ok) drain(0, 1 + grp, drain_parts);  // the CTA's tail
     } else if (warp >= PF_EPI_WARP0 && warp < PF_EPI_WARP0 + 4) {
         // epilogue warps: part 0 of every M-tile's drain
-        for (int mt = 0; mt < nmt && alive; ++mt) alive = drain(mt, 0, C::DRAIN_PARTS);
+        for (int mt = 0; mt < nmt && alive; ++mt) alive = drain(mt, 0, drain_parts);
     }
     tc_fence_before();
     __syncthreads();

@@ -64,12 +64,13 @@ struct PfCfg {
     static constexpr int NISSUE = NMAT;                          // MMA-issuing threads, one per matrix
     // arrivals on a matrix's A slot: one dequant warp per (TMEM lane quadrant, half of the stage)
     static constexpr int DQ_ARRIVALS = 8;
-    // The 4 epilogue warps drain the accumulators.  When a GEMM1 CTA has a
-    // single M-tile, its drain is the CTA's tail and the 16 dequant warps, done
-    // by then, take part: 5 warps per TMEM lane quadrant.  (Joining drains
-    // in the middle of the dequant loop made GEMM1 slower: the drain's
-    // registers spilled there.)
-    static constexpr int SHARED_DRAIN_PARTS = 1 + PF_DQ_THREADS / 128;
+    // The 4 epilogue warps drain the accumulators.  The last M-tile's drain is
+    // the CTA's tail: the 16 dequant warps, done by then, take part (5 warps
+    // per TMEM lane quadrant; only the epilogue warps arrive on "drained",
+    // which nothing waits for after the last M-tile).  (Joining drains in the
+    // middle of the dequant loop made GEMM1 slower: the drain's registers
+    // spilled there.)
+    static constexpr int TAIL_DRAIN_PARTS = 1 + PF_DQ_THREADS / 128;
     static constexpr int B_BYTES = PF_BN_MAX * PF_BK * 2;        // activation tile
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = TSTAGES * B_BYTES + 1024 /*align*/ + PF_BN_MAX * 4 /*gate weights*/ + BAR_BYTES;
@@ -205,8 +206,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         return;
     }
 
-    const bool shared_drain = MODE == 0 && nmt == 1;
-    const int drain_parts = shared_drain ? C::SHARED_DRAIN_PARTS : 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::TSTAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -218,7 +217,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&accf[b], C::NISSUE);
-            mbar_init(&acce[b], shared_drain ? 4 + PF_DQ_THREADS / 32 : 4);
+            mbar_init(&acce[b], 4);
         }
         fence_mbar_init();
     }
@@ -240,7 +239,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // Lane l holds output feature 32 q + l of the M-tile; neighbouring lanes
     // swap values so that each stores a bf16 pair: the even lane features
     // (l, l + 1) of row j, the odd lane features (l - 1, l) of row j + 1.
-    auto drain = [&](int mt, int part, int nparts) -> bool {
+    auto drain = [&](int mt, int part, int nparts, bool arrive) -> bool {
         const int q = warp & 3, odd = lane & 1;
         const int buf = mt % C::NACC, use = mt / C::NACC;
         if (!mbar_wait_fast(&accf[buf], use & 1)) return false;
@@ -289,7 +288,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acce[buf]);
+        if (arrive && lane == 0) mbar_arrive(&acce[buf]);
         return true;
     };
 
@@ -424,10 +423,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (t + 3 >= ntake || !(ok = step(t + 3, p3))) break;
             fetch(t + 7, p3);
         }
-        if (shared_drain && ok) drain(0, 1 + grp, drain_parts);  // the CTA's tail
+        if (ok) drain(nmt - 1, 1 + grp, C::TAIL_DRAIN_PARTS, false);  // the CTA's tail
     } else if (warp >= PF_EPI_WARP0 && warp < PF_EPI_WARP0 + 4) {
         // epilogue warps: part 0 of every M-tile's drain
-        for (int mt = 0; mt < nmt && alive; ++mt) alive = drain(mt, 0, drain_parts);
+        for (int mt = 0; mt < nmt && alive; ++mt)
+            alive = drain(mt, 0, mt == nmt - 1 ? C::TAIL_DRAIN_PARTS : 1, true);
     }
     tc_fence_before();
     __syncthreads();

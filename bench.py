@@ -3,13 +3,19 @@
 
 Headline (one JSON line on rank 0): MoE-layer tokens/s for a decode window of
 T = 5 tokens (1 token + 4 speculative drafts) on a layer of E = 512 experts,
-k = 10, H = 2048, I = 512, 4-bit block-32 weights.  A "prefill" object in the
-same line reports the 8,192-token chunk on the same layer shape.  A step is
-one full layer call (router, grouping, expert FFN, combine, histogram).
+k = 10, H = 2048, I = 512, 4-bit block-32 weights.  Objects in the same line
+report the other workloads, each with its own roofline:
+  decode_T1      the same layer shape, T = 1;
+  prefill        one 8,192-token chunk, 4-bit, Gaussian router;
+  decode_stack   48 layers x 256 experts, 2/2/4-bit, Zipf router, T = 5, chained;
+  prefill_stack  48 layers x 512 experts, 2/2/4-bit, Zipf router, T = 8,192, chained,
+                 with the per-expert roofline sum_e max(flops_e / TC, bytes_e / HBM).
+A step is one full layer call (router, grouping, expert FFN, combine,
+histogram), or one pass through the 48-layer stack for the stacks.
 
-Weights never come from L2: decode steps rotate through 8 layer arenas
-(8 x 906 MB) with a fresh input per layer, prefill through 2 (each 906 MB of
-weights streamed per step, far above the 126 MB L2).
+Weights never come from L2: single-layer workloads rotate through several
+layer arenas (8 x 906 MB for decode, 2 for prefill) with a fresh input per
+layer; a stack step streams 48 layers' experts (GBs) before it repeats.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -33,6 +39,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s (decode T=5, prefill T=8192); % HBM / tensor-pipe roofline"
 DECODE_LAYERS = 8
 PREFILL_LAYERS = 2
+DECODE_WORKLOAD = "decode window: 1 layer, E=512, top_k=10, H=2048, I=512, T=5, 4-bit block-32"
 
 
 def parse():
@@ -42,11 +49,13 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
-    p.add_argument("--no-decode", action="store_true", help="profiling runs: prefill only")
+    p.add_argument("--no-decode", action="store_true", help="profiling runs: no decode sections")
+    p.add_argument("--no-stacks", action="store_true", help="skip the two 48-layer stacks")
     p.add_argument("--no-cpu-baseline", action="store_true", help="profiling runs: skip the oracle timing")
     p.add_argument("--decode-layers", type=int, default=DECODE_LAYERS,
                    help="rotating decode layer arenas (profiling runs use 1)")
     p.add_argument("--prefill-steps", type=int, default=None)
+    p.add_argument("--stack-steps", type=int, default=None)
     return p.parse_args()
 
 
@@ -54,12 +63,11 @@ def profiled_traffic(summary: str, sources) -> int | None:
     """DRAM bytes per launch from a committed ncu summary under profiles/, or None
     when the kernel's sources changed since that capture."""
     import hashlib
-    root = os.path.dirname(os.path.abspath(__file__))
     try:
-        text = open(os.path.join(root, "profiles", summary)).read()
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
         m = hashlib.sha256()
         for f in sources:
-            m.update(open(os.path.join(root, "quantized_expert_ffn_top10_b200", "csrc", f), "rb").read())
+            m.update(open(os.path.join(ROOT, "quantized_expert_ffn_top10_b200", "csrc", f), "rb").read())
         fields = dict(l.split(": ", 1) for l in text.splitlines() if l.startswith(("traffic_", "kernel_sources")))
         if fields.get("kernel_sources_sha256", "").strip() != m.hexdigest():
             return None
@@ -124,18 +132,17 @@ class Clocks:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
-# ----------------------------------------------------------------------------- our arm
+# ----------------------------------------------------------------------------- workloads
 
-class Layers:
-    """NL seeded layers of one shape on the device, each with its own router,
-    input and output; arena slots for layer l are slot_table[l]."""
+class Inputs:
+    """NL seeded layers of one shape on the device (arena, slot table, router,
+    bias, one input per layer).  Uses moe_synth and torch only."""
 
     def __init__(self, cfg, NL: int, rank: int):
         import numpy as np
         import torch
         import moe_synth as S
-        import quantized_expert_ffn_top10_b200 as M
-        self.cfg = S.config(cfg.name, L=NL, seed=replica_seed(cfg.seed, rank))
+        self.cfg = S.config(cfg.name, L=NL, T=cfg.T, seed=replica_seed(cfg.seed, rank))
         c = self.cfg
         self.NL = NL
         self.desc = c.desc()
@@ -145,19 +152,40 @@ class Layers:
         self.b = [None if S.gen_bias(c, l) is None else torch.from_numpy(S.gen_bias(c, l)).cuda() for l in range(NL)]
         self.x_host = [S.gen_x(c, c.T, stream_offset=l) for l in range(NL)]
         self.x = [torch.from_numpy(h.view(np.int16)).cuda() for h in self.x_host]
+
+
+class Layers(Inputs):
+    """Inputs plus what a call through the library needs: workspace, outputs,
+    the histogram and per-layer expert offsets."""
+
+    def __init__(self, cfg, NL: int, rank: int):
+        import torch
+        import quantized_expert_ffn_top10_b200 as M
+        super().__init__(cfg, NL, rank)
+        c = self.cfg
         self.out = [torch.empty_like(v) for v in self.x]
         self.ws = torch.empty(M.moe_workspace_bytes(c.T, c.E, c.top_k, c.H, c.I), dtype=torch.uint8, device="cuda")
         self.hist = torch.zeros((NL, c.E), dtype=torch.int32, device="cuda")
-        P = c.T * c.top_k
         self.offsets = [torch.zeros(c.E + 1, dtype=torch.int32, device="cuda") for _ in range(NL)]
         self.fn = M.moe_forward_prefill if c.T > M.MOE_DECODE_MAX_T else M.moe_forward_decode
-        self.P = P
 
     def call(self, l: int, x=None, out=None):
         c = self.cfg
         self.fn(self.desc, self.arena, self.table, self.NL, l, self.x[l] if x is None else x, self.W[l], self.b[l],
                 c.top_k, True, self.out[l] if out is None else out, hist=self.hist,
                 route_out={"expert_offsets": self.offsets[l]}, ws=self.ws)
+
+    def call_stack(self, a, b):
+        """Layers 0..NL-1 chained: layer l reads one buffer and writes the other."""
+        bufs = (a, b)
+        for l in range(self.NL):
+            self.call(l, x=bufs[l % 2], out=bufs[(l + 1) % 2])
+
+    def distinct(self):
+        return [int((o[1:] - o[:-1] > 0).sum().item()) for o in self.offsets]
+
+    def loads(self):
+        return [(o[1:] - o[:-1]).cpu().numpy() for o in self.offsets]
 
 
 def time_graphs(layers: Layers, steps: int, warmup: int, dev: int, dist):
@@ -184,8 +212,25 @@ def time_graphs(layers: Layers, steps: int, warmup: int, dev: int, dist):
             evs.append(ev)
     M.moe_set_stage_events([])
     torch.cuda.current_stream().wait_stream(s)
+    ms, clk = replay(graphs, steps, warmup, dev, dist)
+    # stage durations of each graph's last replay (all inside the timed region when steps >= NL)
+    try:
+        stages = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]
+    except Exception as ex:  # keep the headline even if the stage hook fails
+        print(f"stage events unavailable: {ex}", file=sys.stderr)
+        stages = [[float("nan")] * 4 for _ in evs]
+    distinct = layers.distinct()
+    del graphs
+    return ms, stages, distinct, per_call, clk
+
+
+def replay(graphs, steps: int, warmup: int, dev: int, dist):
+    """Warm-up replays, then `steps` timed replays round-robin between a
+    barrier and a synchronize on each side; CUDA events, max over ranks."""
+    import torch
+    n = len(graphs)
     for i in range(warmup):
-        graphs[i % NL].replay()
+        graphs[i % n].replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -194,22 +239,35 @@ def time_graphs(layers: Layers, steps: int, warmup: int, dev: int, dist):
     with Clocks(dev) as clk:
         e0.record()
         for i in range(steps):
-            graphs[(warmup + i) % NL].replay()
+            graphs[(warmup + i) % n].replay()
         e1.record()
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if dist:
         dist.barrier()
-    ms = max_over_ranks(dist, ms)
-    # stage durations of each graph's last replay (all inside the timed region when steps >= NL)
-    try:
-        stages = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]
-    except Exception as ex:  # keep the headline even if the stage hook fails
-        print(f"stage events unavailable: {ex}", file=sys.stderr)
-        stages = [[float("nan")] * 4 for _ in evs]
-    distinct = [int((layers.offsets[l][1:] - layers.offsets[l][:-1] > 0).sum().item()) for l in range(NL)]
-    del graphs
-    return ms, stages, distinct, per_call, clk.summary()
+    return max_over_ranks(dist, ms), clk.summary()
+
+
+def time_stack(layers: Layers, steps: int, warmup: int, dev: int, dist):
+    """One graph holding the whole chained stack; replayed `steps` times."""
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    a = layers.x[0].clone()
+    b = torch.empty_like(a)
+    n0 = M.moe_launch_count()
+    layers.call_stack(a.clone(), b)  # eager pass: one-time init, launches per step
+    torch.cuda.synchronize()
+    per_step = M.moe_launch_count() - n0
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            layers.call_stack(a, b)
+    torch.cuda.current_stream().wait_stream(s)
+    ms, clk = replay([g], steps, warmup, dev, dist)
+    del g
+    return ms, per_step, clk
 
 
 def time_e2e(layers: Layers, steps: int, warmup: int, dist):
@@ -246,33 +304,45 @@ def time_e2e(layers: Layers, steps: int, warmup: int, dist):
 
 # ----------------------------------------------------------------------------- oracle (CPU baseline / reference arm)
 
-def oracle_sample(layers: Layers, l: int, n_tokens: int):
+def oracle_sample(inp, l: int, n_tokens: int, host_slots: bool = False):
     """Run the CPU oracle on the first n_tokens of layer l's input (router over
     every expert, then the selected experts' FFNs and the combine); returns
-    (seconds, tokens).  Slots are read from the generated arena in HBM."""
+    (seconds, tokens).  Slots come from the arena in HBM, or (host_slots) are
+    regenerated on the host from the workload's seeded streams."""
     import numpy as np
     import moe_synth as S
     import oracle as O
-    c = layers.cfg
-    x = layers.x_host[l][:n_tokens]
-    W = layers.W[l].cpu().numpy()
-    b = None if layers.b[l] is None else layers.b[l].cpu().numpy()
-    table = layers.table.cpu().numpy()
-    sb = layers.desc.slot_bytes
-    lg = O.router_logits(x, W, b)  # untimed: only to know which slots to copy to the host
+    c = inp.cfg
+    x = inp.x_host[l][:n_tokens]
+    W = inp.W[l] if isinstance(inp.W[l], np.ndarray) else inp.W[l].cpu().numpy()
+    b = inp.b[l]
+    if b is not None and not isinstance(b, np.ndarray):
+        b = b.cpu().numpy()
+    table = inp.table if isinstance(inp.table, np.ndarray) else inp.table.cpu().numpy()
+    sb = inp.desc.slot_bytes
+    lg = O.router_logits(x, W, b)  # untimed: only to know which slots to gather
     idx, _ = O.topk(lg, c.top_k)
     ex = sorted(set(idx.reshape(-1).tolist()))
     mini = np.zeros(len(ex) * sb, np.uint8)
     mt = np.full(c.L * c.E, -1, np.int32)
     for i, e in enumerate(ex):
         s = int(table[l * c.E + e])
-        mini[i * sb:(i + 1) * sb] = layers.arena[s * sb:(s + 1) * sb].cpu().numpy()
+        mini[i * sb:(i + 1) * sb] = S.gen_slot_host(c, s) if host_slots else inp.arena[s * sb:(s + 1) * sb].cpu().numpy()
         mt[l * c.E + e] = i
     d = S.make_desc(c.H, c.I, c.bits, n_slots=len(ex))
     t1 = time.perf_counter()
     O.moe_layer(d, mini, mt, c.L, l, x, W, b, c.top_k)  # routes again, then the FFNs
-    t_layer = time.perf_counter() - t1
-    return t_layer, n_tokens
+    return time.perf_counter() - t1, n_tokens
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def cores():
@@ -280,6 +350,22 @@ def cores():
         return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
+
+
+def cpu_baseline(inp, l: int, n_tokens: int, sample: str, host_slots: bool = False) -> dict:
+    """The oracle as it stands on this host: all cores (its OpenMP loops over
+    tokens and pairs) and one thread, on the same bounded sample."""
+    import oracle as O
+    allc = O.max_threads()
+    secs, n = oracle_sample(inp, l, n_tokens, host_slots)
+    O.set_threads(1)
+    try:
+        secs1, _ = oracle_sample(inp, l, n_tokens, host_slots)
+    finally:
+        O.set_threads(allc)
+    return {"value": round(n / secs, 3), "unit": "tokens/s", "cores": allc, "kind": "oracle", "sample": sample,
+            "single_thread": {"value": round(n / secs1, 3), "unit": "tokens/s", "cores": 1},
+            "cpu_model": cpu_model(), "host_cpus": cores()}
 
 
 # ----------------------------------------------------------------------------- main
@@ -319,16 +405,27 @@ def decode_bytes(c, distinct: int):
 
 
 def gateup_bytes(c, distinct: int):
-    d = c.desc()
     per = 0
     for m in (0, 1):
         per += c.I * c.H * c.bits[m] // 8 + c.I * (c.H // 32) * 2
     return distinct * per + c.T * c.H * 2 + c.T * c.top_k * c.I * 4
 
 
+def prefill_min_ms(c, loads, hbm_gbs: float, tc_tflops: float) -> float:
+    """Per-expert roofline of one prefill layer: sum over experts with pairs of
+    max(flops_e / tensor peak, bytes_e / HBM peak), plus the router's
+    max(flops / tensor peak, (router weights + x in + out) / HBM peak), in ms."""
+    sb = c.desc().slot_bytes
+    t = 0.0
+    for n in loads:
+        if n > 0:
+            t = t + max(6.0 * n * c.H * c.I / (tc_tflops * 1e9), sb / (hbm_gbs * 1e6))
+    t += max(2.0 * c.T * c.E * c.H / (tc_tflops * 1e9), (c.E * c.H * 4 + 4 * c.T * c.H) / (hbm_gbs * 1e6))
+    return t
+
+
 def run_ours(args):
     import torch
-    import moe_synth as S
     rank, local, world = rank_env()
     torch.cuda.set_device(local)
     dist = None
@@ -337,24 +434,20 @@ def run_ours(args):
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = tdist
-    hbm, tc_burst, tc_sus, src = peaks()
+    pk = peaks()
     K, W = args.steps, max(3, args.warmup)
-
+    base = rank == 0 and world == 1 and not args.no_cpu_baseline
     line = {"metric": METRIC}
-    if args.no_decode:
-        run_prefill_only = True
-    else:
-        run_prefill_only = False
-    # ---- decode (headline)
-    if not run_prefill_only:
-        line = decode_section(args, rank, local, world, dist, hbm, src, K, W)
-    prefill_section(args, line, rank, local, world, dist, tc_burst, tc_sus, src, K, W)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not run_prefill_only:
-        dl = Layers(S.config("decode"), 1, rank)
-        secs, n = oracle_sample(dl, 0, 5)
-        line["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores(), "kind": "oracle",
-                                "sample": "one decode window (T=5) of one layer: router over 512 experts, "
-                                          "the selected experts' FFNs, combine"}
+    if not args.no_decode:
+        line = decode_section(args, rank, local, world, dist, pk, K, W, base)
+        line["decode_T1"] = decode_t1_section(args, rank, local, world, dist, pk, K, W, base)
+    if not args.no_prefill:
+        prefill_section(args, line, rank, local, world, dist, pk, K, W, base)
+    if not args.no_stacks:
+        if not args.no_decode:
+            line["decode_stack"] = decode_stack_section(args, rank, local, world, dist, pk, W, base)
+        if not args.no_prefill:
+            line["prefill_stack"] = prefill_stack_section(args, rank, local, world, dist, pk, W, base)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -362,9 +455,15 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def decode_section(args, rank, local, world, dist, hbm, src, K, W):
+DECODE_DTYPE = ("u4/u2 codes; decode: bf16 x bf16 mma.sync on exact (128 + code) and x, fp32 accumulation, "
+                "scales applied in fp32, h rounded to bf16; prefill: bf16 tcgen05 MMA on dequantised weights, "
+                "fp32 accumulation in TMEM, h and per-pair outputs in bf16; output bf16")
+
+
+def decode_section(args, rank, local, world, dist, pk, K, W, base):
     import torch
     import moe_synth as S
+    hbm, _, _, src = pk
     NLd = max(1, args.decode_layers)
     dl = Layers(S.config("decode"), NLd, rank)
     c = dl.cfg
@@ -378,9 +477,9 @@ def decode_section(args, rank, local, world, dist, hbm, src, K, W):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms / K, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u4 codes, fp32 math (decode); bf16 tensor-core MMA, fp32 accumulate (prefill)",
+        "dtype": DECODE_DTYPE,
         "data": "synthetic (seeded; random-init weights of the stated shape)",
-        "config": {"workload": "decode window: 1 layer, E=512, top_k=10, H=2048, I=512, T=5, 4-bit block-32",
+        "config": {"workload": DECODE_WORKLOAD,
                    "l2": f"{NLd} rotating layer arenas ({NLd * 0.906:.1f} GB) with fresh inputs",
                    "graph": "one CUDA graph per layer call", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": "k_decode_fused (whole layer)" if fused else "decode gate/up + SwiGLU",
@@ -401,70 +500,174 @@ def decode_section(args, rank, local, world, dist, hbm, src, K, W):
         "gpu_launches": per_call * K,
         "clocks": clk,
     }
+    if base:
+        line["cpu_baseline"] = cpu_baseline(dl, 0, 5, "one decode window (T=5) of one layer: router over 512 "
+                                                      "experts, the selected experts' FFNs, combine")
     del dl
     torch.cuda.empty_cache()
     return line
 
 
-def prefill_section(args, line, rank, local, world, dist, tc_burst, tc_sus, src, K, W):
+def decode_t1_section(args, rank, local, world, dist, pk, K, W, base):
     import torch
     import moe_synth as S
-    if not args.no_prefill:
-        pl = Layers(S.config("prefill"), PREFILL_LAYERS, rank)
-        cp = pl.cfg
-        Kp = args.prefill_steps or max(PREFILL_LAYERS, min(K, 20))
-        msp, stp, dsp, pcp, clkp = time_graphs(pl, Kp, W, local, dist)
-        P = cp.T * cp.top_k
-        g1 = statistics.mean(s[1] for s in stp)
-        g2 = statistics.mean(s[2] for s in stp)
-        f1 = 4.0 * P * cp.H * cp.I
-        f2 = 2.0 * P * cp.H * cp.I
-        flops = f1 + f2 + 2.0 * cp.T * cp.E * cp.H
-        e2p, h2p, d2p = time_e2e(pl, max(2, Kp // 4), 2, dist)
-        line["prefill"] = {
-            "value": round(whole_job_rate(cp.T * Kp, world, msp), 1), "unit": "tokens/s", "steps": Kp,
-            "ms_per_step": round(msp / Kp, 4),
-            "workload": "prefill chunk: 1 layer, E=512, top_k=10, H=2048, I=512, T=8192, 4-bit, Gaussian router",
-            "roofline": {"bound": "tensor", "kernel": "prefill gate/up grouped GEMM + SwiGLU",
-                         "achieved": round(f1 / (g1 * 1e9), 1), "peak": tc_sus, "unit": "TFLOP/s",
-                         "frac": round(f1 / (g1 * 1e9) / tc_sus, 4),
-                         "traffic": profiled_traffic("k_prefill_gemm_prefill_T8192.md", ("common.cuh", "prefill.cuh")),
-                         "peak_source": src + " sustained",
-                         "ms": round(g1, 4)},
-            "gemm2": {"achieved": round(f2 / (g2 * 1e9), 1), "unit": "TFLOP/s", "frac": round(f2 / (g2 * 1e9) / tc_sus, 4),
-                      "ms": round(g2, 4)},
-            "layer_tc_frac": round(flops / (msp / Kp * 1e9) / tc_sus, 4),
-            "layer_tc_frac_burst": round(flops / (msp / Kp * 1e9) / tc_burst, 4),
-            "stage_ms": [round(statistics.mean(s[j] for s in stp), 4) for j in range(4)],
-            "e2e": {"value": round(whole_job_rate(cp.T * max(2, Kp // 4), world, e2p), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2p, "d2h_bytes_per_step": d2p},
-            "gpu_launches": pcp * Kp, "clocks": clkp,
-        }
-        line["gpu_launches"] = line.get("gpu_launches", 0) + pcp * Kp
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            secs, n = oracle_sample(pl, 0, 16)
-            line["prefill"]["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores(),
-                                               "kind": "oracle",
-                                               "sample": "16 tokens of the 8,192-token chunk, full layer"}
-        del pl
-        torch.cuda.empty_cache()
+    hbm, _, _, src = pk
+    NLd = max(1, args.decode_layers)
+    dl = Layers(S.config("decode", T=1), NLd, rank)
+    c = dl.cfg
+    ms, stages, distinct, per_call, clk = time_graphs(dl, K, W, local, dist)
+    kern = statistics.mean(s[0] + s[1] + s[2] + s[3] for s in stages)
+    nbytes = statistics.mean(decode_bytes(c, d) for d in distinct)
+    sec = {"value": round(whole_job_rate(c.T * K, world, ms), 1), "unit": "tokens/s", "steps": K,
+           "ms_per_step": round(ms / K, 5),
+           "workload": "decode, 1 token: 1 layer, E=512, top_k=10, H=2048, I=512, T=1, 4-bit block-32",
+           "roofline": {"bound": "hbm", "kernel": "k_decode_fused (whole layer)" if per_call == 1 else "decode layer",
+                        "achieved": round(nbytes / (kern * 1e6), 1), "peak": hbm, "unit": "GB/s",
+                        "frac": round(nbytes / (kern * 1e6) / hbm, 4), "peak_source": src, "ms": round(kern, 5),
+                        "bytes": int(nbytes), "distinct_experts": statistics.mean(distinct)},
+           "layer_frac": round(nbytes / (ms / K * 1e6) / hbm, 4),
+           "gpu_launches": per_call * K, "clocks": clk}
+    if base:
+        sec["cpu_baseline"] = cpu_baseline(dl, 0, 1, "one decode token (T=1) of one layer")
+    del dl
+    torch.cuda.empty_cache()
+    return sec
+
+
+def prefill_section(args, line, rank, local, world, dist, pk, K, W, base):
+    import torch
+    import moe_synth as S
+    hbm, tc_burst, tc_sus, src = pk
+    pl = Layers(S.config("prefill"), PREFILL_LAYERS, rank)
+    cp = pl.cfg
+    Kp = args.prefill_steps or max(PREFILL_LAYERS, min(K, 20))
+    msp, stp, dsp, pcp, clkp = time_graphs(pl, Kp, W, local, dist)
+    P = cp.T * cp.top_k
+    g1 = statistics.mean(s[1] for s in stp)
+    g2 = statistics.mean(s[2] for s in stp)
+    f1 = 4.0 * P * cp.H * cp.I
+    f2 = 2.0 * P * cp.H * cp.I
+    flops = f1 + f2 + 2.0 * cp.T * cp.E * cp.H
+    e2p, h2p, d2p = time_e2e(pl, max(2, Kp // 4), 2, dist)
+    step_ms = msp / Kp
+    line["prefill"] = {
+        "value": round(whole_job_rate(cp.T * Kp, world, msp), 1), "unit": "tokens/s", "steps": Kp,
+        "ms_per_step": round(step_ms, 4),
+        "workload": "prefill chunk: 1 layer, E=512, top_k=10, H=2048, I=512, T=8192, 4-bit, Gaussian router",
+        "roofline": {"bound": "tensor", "kernel": "prefill gate/up grouped GEMM + SwiGLU",
+                     "achieved": round(f1 / (g1 * 1e9), 1), "peak": tc_burst, "unit": "TFLOP/s",
+                     "frac": round(f1 / (g1 * 1e9) / tc_burst, 4),
+                     "traffic": profiled_traffic("k_prefill_gemm_prefill_T8192.md", ("common.cuh", "prefill.cuh")),
+                     "peak_source": src + " burst (a ~1 ms step, a timed region of tens of ms)",
+                     "ms": round(g1, 4)},
+        "gemm2": {"achieved": round(f2 / (g2 * 1e9), 1), "unit": "TFLOP/s", "frac": round(f2 / (g2 * 1e9) / tc_burst, 4),
+                  "ms": round(g2, 4)},
+        "layer_tc_frac": round(flops / (step_ms * 1e9) / tc_burst, 4),
+        "layer_tc_frac_sustained": round(flops / (step_ms * 1e9) / tc_sus, 4),
+        "stage_ms": [round(statistics.mean(s[j] for s in stp), 4) for j in range(4)],
+        "e2e": {"value": round(whole_job_rate(cp.T * max(2, Kp // 4), world, e2p), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2p, "d2h_bytes_per_step": d2p},
+        "gpu_launches": pcp * Kp, "clocks": clkp,
+    }
+    if base:
+        line["prefill"]["cpu_baseline"] = cpu_baseline(pl, 0, 16, "16 tokens of the 8,192-token chunk, full layer")
+    del pl
+    torch.cuda.empty_cache()
+
+
+def decode_stack_section(args, rank, local, world, dist, pk, W, base):
+    import torch
+    import moe_synth as S
+    hbm, _, _, src = pk
+    st = Layers(S.config("decode_stack"), 48, rank)
+    c = st.cfg
+    Ks = args.stack_steps or 20
+    ms, per_step, clk = time_stack(st, Ks, W, local, dist)
+    distinct = st.distinct()  # of the last replay (the same input every step)
+    nbytes = sum(decode_bytes(c, d) for d in distinct)
+    step_ms = ms / Ks
+    sec = {"value": round(whole_job_rate(c.T * c.L * Ks, world, ms), 1), "unit": "token-layers/s",
+           "tokens_per_s_through_stack": round(whole_job_rate(c.T * Ks, world, ms), 1), "steps": Ks,
+           "ms_per_step": round(step_ms, 4), "ms_per_layer": round(step_ms / c.L, 5),
+           "workload": "pruned decode stack: 48 layers x E=256, top_k=10, H=2048, I=512, T=5, gate/up 2-bit, "
+                       "down 4-bit, Zipf(1.1) router bias, residual chain",
+           "roofline": {"bound": "hbm", "achieved": round(nbytes / (step_ms * 1e6), 1), "peak": hbm, "unit": "GB/s",
+                        "frac": round(nbytes / (step_ms * 1e6) / hbm, 4), "peak_source": src,
+                        "bytes_per_step": int(nbytes), "distinct_experts_mean": round(statistics.mean(distinct), 2),
+                        "distinct_experts_max": max(distinct)},
+           "gpu_launches": per_step * Ks, "clocks": clk,
+           "l2": "a step streams 48 layers' selected experts from a 15.3 GB arena"}
+    if base:
+        sec["cpu_baseline"] = cpu_baseline(st, 0, 5, "one T=5 window through layer 0 of the stack")
+    del st
+    torch.cuda.empty_cache()
+    return sec
+
+
+def prefill_stack_section(args, rank, local, world, dist, pk, W, base):
+    import torch
+    import moe_synth as S
+    hbm, tc_burst, tc_sus, src = pk
+    st = Layers(S.config("prefill_stack"), 48, rank)
+    c = st.cfg
+    Ks = args.stack_steps or 6
+    ms, per_step, clk = time_stack(st, Ks, W, local, dist)
+    loads = st.loads()
+    step_ms = ms / Ks
+    flops = c.L * (6.0 * c.T * c.top_k * c.H * c.I + 2.0 * c.T * c.E * c.H)
+    tmin_b = sum(prefill_min_ms(c, ld, hbm, tc_burst) for ld in loads)
+    tmin_s = sum(prefill_min_ms(c, ld, hbm, tc_sus) for ld in loads)
+    nz = [int((ld > 0).sum()) for ld in loads]
+    sec = {"value": round(whole_job_rate(c.T * c.L * Ks, world, ms), 1), "unit": "token-layers/s",
+           "tokens_per_s_through_stack": round(whole_job_rate(c.T * Ks, world, ms), 1), "steps": Ks,
+           "ms_per_step": round(step_ms, 3), "ms_per_layer": round(step_ms / c.L, 4),
+           "workload": "prefill stack: 48 layers x E=512, top_k=10, H=2048, I=512, T=8192, gate/up 2-bit, down 4-bit, "
+                       "Zipf(1.1) router bias, residual chain; outputs plus the 48 x 512 histogram",
+           "roofline": {"bound": "per-expert max(tensor, hbm)", "t_min_ms": round(tmin_b, 3),
+                        "frac": round(tmin_b / step_ms, 4), "frac_sustained_tc": round(tmin_s / step_ms, 4),
+                        "peak_tc": tc_burst, "peak_hbm": hbm, "peak_source": src + " burst tensor, copy HBM",
+                        "dense_tc_frac": round(flops / (step_ms * 1e9) / tc_burst, 4)},
+           "loads": {"max_pairs_per_expert": int(max(ld.max() for ld in loads)),
+                     "experts_used_min": min(nz), "experts_used_mean": round(statistics.mean(nz), 1)},
+           "gpu_launches": per_step * Ks, "clocks": clk}
+    if base:
+        sec["cpu_baseline"] = cpu_baseline(st, 0, 16, "16 tokens through layer 0 of the stack")
+    del st
+    torch.cuda.empty_cache()
+    return sec
+
+
+class HostInputs:
+    """The reference arm's inputs on the host only (moe_synth; no GPU and no
+    part of the library): x, router and bias of each layer, the slot table;
+    slots are regenerated from their seeded streams when the oracle needs them."""
+
+    def __init__(self, cfg, NL: int):
+        import moe_synth as S
+        self.cfg = S.config(cfg.name, L=NL, T=cfg.T, seed=cfg.seed)
+        c = self.cfg
+        self.NL = NL
+        self.desc = c.desc()
+        self.table = S.gen_slot_table(c)
+        self.W = [S.gen_router(c, l) for l in range(NL)]
+        self.b = [S.gen_bias(c, l) for l in range(NL)]
+        self.x_host = [S.gen_x(c, c.T, stream_offset=l) for l in range(NL)]
 
 
 def run_reference(args):
     """The oracle as the reference arm: each step is one decode window (T=5)
-    of a seeded layer on the host cores."""
+    of a seeded layer, on the host cores of rank 0."""
     rank, local, world = rank_env()
     if rank != 0:
         return
-    import torch
     import moe_synth as S
-    torch.cuda.set_device(local)
-    dl = Layers(S.config("decode"), 2, 0)
+    import oracle as O
+    inp = HostInputs(S.config("decode"), 2)
     for i in range(args.warmup):
-        oracle_sample(dl, i % 2, 5)
+        oracle_sample(inp, i % 2, 5, host_slots=True)
     tot, n = 0.0, 0
     for i in range(args.steps):
-        s, t = oracle_sample(dl, i % 2, 5)
+        s, t = oracle_sample(inp, i % 2, 5, host_slots=True)
         tot += s
         n += t
     v = n / tot
@@ -472,10 +675,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp64 (CPU oracle)",
-        "data": "synthetic", "config": {"workload": "decode window: 1 layer, E=512, top_k=10, H=2048, I=512, T=5, "
-                                                    "4-bit block-32"},
-        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": cores(), "kind": "oracle",
-                         "sample": "each step one decode window (T=5) of one layer"},
+        "data": "synthetic", "config": {"workload": DECODE_WORKLOAD},
+        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": O.max_threads(), "kind": "oracle",
+                         "sample": "each step one decode window (T=5) of one layer", "cpu_model": cpu_model()},
         "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

@@ -106,7 +106,13 @@ typedef struct moe_route_out {
 size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I);
 
 /*
- * Router and grouping only.
+ * Router and grouping only.  Defined by the "Strata Coder deep-dive" page,
+ * section 1 (each token of a layer is routed to 10 of its 512 experts, 256 in
+ * the pruned variant of section 2), and the "Coder benchmark record" page,
+ * "why Coder is fast" (experts addressed and fetched per (layer, expert)):
+ * logits l = x W_r^T + b, the top_k experts by (l desc, e asc) - bit-exact
+ * against the fp64 sequential definition, certified on the device - their
+ * softmax gate weights, and the pairs (t, j) grouped by expert.
  *   x [T][H] bf16 (device, 16-B aligned), router_w [E][H] fp32 (device,
  *   16-B aligned), router_bias [E] fp32 (device) or NULL.
  *   Outputs (device): topk_idx [T*k], topk_w [T*k], expert_offsets [E+1],
@@ -120,10 +126,13 @@ int moe_route(const uint16_t* x, int T, int H, const float* router_w, const floa
 /*
  * moe_route without a caller workspace: the same router and grouping kernels,
  * with their scratch in a fixed device array inside libmoe.so
- * (MOE_ROUTE_STATIC_BYTES per device, located once per device with
- * cudaGetSymbolAddress).  No page of the method has a counterpart: it is a
- * serving convenience for callers that cannot hand over a workspace, and it
- * allocates nothing (no cudaMalloc, no cudaFree, no allocator of any kind).
+ * (MOE_ROUTE_STATIC_BYTES per device; every GPU that loads the library holds
+ * it until the process exits).  No page of the method has a counterpart: it
+ * is a serving convenience for callers that cannot hand over a workspace, and
+ * it allocates nothing (no cudaMalloc, no cudaFree, no allocator of any kind).
+ * The array's device address is looked up with cudaGetSymbolAddress by the
+ * first call in each CUDA context of a device (again after cudaDeviceReset or
+ * under another context); make that first call before any stream capture.
  *   Arguments, layouts and outputs as moe_route.  Limits: 1 <= T <=
  *   MOE_ROUTE_STATIC_MAX_T, 1 <= E <= 512, 1 <= top_k <= min(E, 32); a T
  *   above the limit returns MOE_ERR_STATIC before any CUDA call.  T = 0 is a
@@ -144,6 +153,12 @@ int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, con
  * Full layer for a decode window, 1 <= T <= MOE_DECODE_MAX_T: router, grouping,
  * fused dequant + SwiGLU gate/up, down projection, weighted combine (+x when
  * residual != 0) and, when hist != NULL, hist[layer][e] += pairs routed to e.
+ * Defined by the "Strata Coder deep-dive" page, sections 1-3 (10 of 512
+ * experts per token; an expert is gate, up and down projections stored
+ * block-quantized at low bit width, gate/up narrower than down) and the
+ * "Coder benchmark record" page, test environment (a verify window of the
+ * token plus 4 speculative drafts, T = 5) and "why Coder is fast" (each
+ * selected expert's weights are read once per window).
  *   desc (host); arena (device, 256-B aligned); slot_table [L][E] int32
  *   (device); x [T][H] bf16 (device); out [T][H] bf16 (device);
  *   hist [L][E] uint32 (device, persistent, caller-owned) or NULL;
@@ -160,7 +175,11 @@ int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int3
  * Full layer for a prefill chunk, 1 <= T <= MOE_PREFILL_MAX_T: same arguments
  * and results as moe_forward_decode; the expert FFN runs as per-expert grouped
  * GEMMs on the tensor cores (weights dequantised to bf16 on chip, SwiGLU
- * output h rounded to bf16, per-pair expert outputs kept in bf16).
+ * output h rounded to bf16, per-pair expert outputs kept in bf16).  Defined
+ * by the same passages as moe_forward_decode, with the chunked prompt path of
+ * the "Coder benchmark record" page, test environment (prompts processed in
+ * chunks of at most 8,192 tokens), and of the "Strata overview" page, chunked
+ * prefill.
  */
 int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
                         int L, int layer, const uint16_t* x, int T, const float* router_w,
@@ -172,7 +191,9 @@ int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int
  * Routing-count histogram ("--dump-routing" counts of the benchmark record
  * page): hist[layer][e] += expert_offsets[e+1] - expert_offsets[e] for
  * e < E, one owner thread per expert, no atomics.  expert_offsets [E+1]
- * (device), hist [L][E] uint32 (device).
+ * (device), hist [L][E] uint32 (device).  The update is a plain read-add-
+ * write: calls (and forward calls with hist != NULL) that add to the same
+ * hist must be ordered, e.g. on one stream; concurrent ones lose counts.
  */
 int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, uint32_t* hist,
                         void* stream);
@@ -207,6 +228,34 @@ const char* moe_strerror(int code);
  */
 int moe_set_stage_events(void* const* events, int n);
 uint64_t moe_launch_count(void);
+
+/*
+ * Test hooks (no counterpart on the source pages; off by default, never used
+ * by the layer itself):
+ * moe_debug_set(MOE_DBG_SPIN_LIMIT, n): grid-barrier waits of the fused decode
+ *   kernel give up after n polls instead of about 2 s worth (0 restores it).
+ * moe_debug_set(MOE_DBG_BARRIER_EXTRA, n): the fused decode kernel's first
+ *   grid barrier waits for n arrivals that never come, so that every CTA
+ *   runs into the polling bound and reports MOE_ERR_TIMEOUT (site 1) with no
+ *   copy in flight and no tensor memory held; 0 restores it.
+ * Both are process-wide and read when a forward call is enqueued.
+ * moe_workspace_offset(T, E, top_k, H, I, field): byte offset inside a forward
+ *   or route workspace of MOE_WS_FAST_LOGITS (the router's fast logits: fp32
+ *   [T][E] for chunks T > MOE_DECODE_MAX_T, fp64 for decode windows) or
+ *   MOE_WS_PAIR_OUT (per-pair expert outputs w * y in pair order: bf16 [T*k][H]
+ *   for chunks); (size_t)-1 for bad arguments.
+ * moe_router_gamma(T, E, H): for a chunk (T > MOE_DECODE_MAX_T), the factor
+ *   gamma of the fast logits' certified bound |fast - exact| <= gamma *
+ *   (||x_t|| ||W_r[e]|| + |b_e|) (before the fp64 definition's own rounding
+ *   term); -1 for decode windows or bad sizes.
+ */
+#define MOE_DBG_SPIN_LIMIT 1
+#define MOE_DBG_BARRIER_EXTRA 2
+#define MOE_WS_FAST_LOGITS 1
+#define MOE_WS_PAIR_OUT 2
+int moe_debug_set(int key, int value);
+size_t moe_workspace_offset(int T, int E, int top_k, int H, int I, int field);
+double moe_router_gamma(int T, int E, int H);
 
 /* Diagnostic companion of MOE_ERR_TIMEOUT: after synchronising `stream`,
  * returns and clears where the first bounded device wait gave up

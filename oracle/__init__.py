@@ -70,6 +70,10 @@ def lib():
         L.oracle_moe_layer.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
                                        ctypes.c_int]
+        L.oracle_set_threads.restype = None
+        L.oracle_set_threads.argtypes = [ctypes.c_int]
+        L.oracle_max_threads.restype = ctypes.c_int
+        L.oracle_max_threads.argtypes = []
         del i32, i64
         _lib = L
     return _lib
@@ -126,6 +130,42 @@ def expert_ffn(slot: np.ndarray, desc, x: np.ndarray):
     h = np.zeros(desc.I, np.float64)
     lib().oracle_expert_ffn(_p(slot), ctypes.byref(desc), _p(x), _p(y), _p(h))
     return y, h
+
+
+def dequant_matrix(slot: np.ndarray, desc, m: int) -> np.ndarray:
+    """Matrix m (0 gate [I, H], 1 up [I, H], 2 down [H, I]) of one slot, fp64:
+    W[r, c] = scale[r, c // 32] * (code[r, c] - 2^(bits - 1)), codes packed
+    LSB first along each row.  The same definition as oracle_dequant (the
+    block-32 reading of the "Strata Coder deep-dive" page, sections 2-3),
+    unpacked for a whole matrix at once."""
+    slot = np.asarray(slot, np.uint8)
+    rows, K = (desc.I, desc.H) if m < 2 else (desc.H, desc.I)
+    b = (desc.bits_gate, desc.bits_up, desc.bits_down)[m]
+    o = desc.off_codes[m]
+    raw = slot[o:o + rows * K * b // 8].astype(np.int64)
+    per = 8 // b
+    codes = np.empty((raw.size, per), np.int64)
+    for i in range(per):                       # element i of a byte sits at bits i*b .. i*b + b - 1
+        codes[:, i] = (raw >> (i * b)) & ((1 << b) - 1)
+    codes = codes.reshape(rows, K)
+    so = desc.off_scales[m]
+    sc = slot[so:so + rows * (K // 32) * 2].view("<f2").astype(np.float64).reshape(rows, K // 32)
+    return np.repeat(sc, 32, axis=1) * (codes - (1 << (b - 1))).astype(np.float64)
+
+
+def expert_ffn_rows(slot: np.ndarray, desc, X: np.ndarray):
+    """(y [n, H], h [n, I]) of one expert for n fp64 token rows X [n, H]:
+    g = W_g x, u = W_u x, h = silu(g) u, y = W_d h - the definition of
+    oracle_expert_ffn (SwiGLU reading of the gate/up/down projections of the
+    "Strata Coder deep-dive" page, section 3), with each matrix dequantised
+    once and the sums taken by numpy's fp64 matrix product, so that thousands
+    of rows of one expert take seconds."""
+    X = np.asarray(X, np.float64)
+    Wg, Wu, Wd = (dequant_matrix(slot, desc, m) for m in range(3))
+    g = X @ Wg.T
+    u = X @ Wu.T
+    h = g / (1.0 + np.exp(-g)) * u
+    return h @ Wd.T, h
 
 
 # --------------------------------------------------------------- routing
@@ -203,3 +243,14 @@ def moe_layer(desc, arena: np.ndarray, slot_table: np.ndarray, L: int, layer: in
                                 _p(x_bits), T, _p(W), _p(b), E, k, int(bool(residual)),
                                 _p(out), _p(out64), _p(idx), _p(w), _p(tok), nt)
     return {"out": out, "out_f64": out64, "idx": idx, "w": w, "rc": rc}
+
+
+# --------------------------------------------------------------- timing control
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops (results do not depend on it)."""
+    lib().oracle_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())

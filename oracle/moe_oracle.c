@@ -35,6 +35,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_ERR_ARG (-1)
@@ -310,4 +313,24 @@ int oracle_moe_layer(const orc_desc* d, const uint8_t* arena, const int32_t* slo
     }
     free(logit); free(xs); free(idx); free(w); free(y);
     return bad_slot ? ORC_ERR_SLOT : ORC_OK;
+}
+
+/* ---------------------------------------------------------------- threads */
+
+/* Threads of the parallel loops over tokens and pairs (a timing control:
+ * every value is computed by one thread in the same order either way). */
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }

@@ -44,7 +44,10 @@ MOE_ROUTE_STATIC_MAX_T, MOE_ROUTE_STATIC_BYTES = 8, 128 * 1024
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",
            "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
-           "moe_set_stage_events", "moe_launch_count", "moe_timeout_site", "moe_route_static")
+           "moe_set_stage_events", "moe_launch_count", "moe_timeout_site", "moe_route_static",
+           "moe_debug_set", "moe_workspace_offset", "moe_router_gamma")
+MOE_DBG_SPIN_LIMIT, MOE_DBG_BARRIER_EXTRA = 1, 2
+MOE_WS_FAST_LOGITS, MOE_WS_PAIR_OUT = 1, 2
 
 
 class RouteOut(ctypes.Structure):
@@ -94,6 +97,12 @@ def lib() -> ctypes.CDLL:
         L.moe_timeout_site.argtypes = [P]
         L.moe_route_static.restype = i32
         L.moe_route_static.argtypes = [P, i32, i32, P, P, i32, i32, P, P, P, P, P]
+        L.moe_debug_set.restype = i32
+        L.moe_debug_set.argtypes = [i32, i32]
+        L.moe_workspace_offset.restype = sz
+        L.moe_workspace_offset.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.moe_router_gamma.restype = ctypes.c_double
+        L.moe_router_gamma.argtypes = [i32, i32, i32]
         _lib = L
     return _lib
 
@@ -216,3 +225,21 @@ def moe_launch_count() -> int:
 
 def moe_timeout_site(stream=None) -> int:
     return int(lib().moe_timeout_site(_stream(stream)))
+
+
+def moe_debug_set(key: int, value: int) -> int:
+    """Test hook: see include/moe.h (MOE_DBG_SPIN_LIMIT, MOE_DBG_BARRIER_EXTRA)."""
+    return _check(lib().moe_debug_set(int(key), int(value)), "moe_debug_set", True)
+
+
+def moe_workspace_offset(T: int, E: int, top_k: int, H: int, I: int, field: int) -> int:
+    """Byte offset of a workspace field (MOE_WS_FAST_LOGITS, MOE_WS_PAIR_OUT)."""
+    v = int(lib().moe_workspace_offset(T, E, top_k, H, I, field))
+    if v == ctypes.c_size_t(-1).value:
+        raise MoeError(MOE_ERR_ARG, "moe_workspace_offset")
+    return v
+
+
+def moe_router_gamma(T: int, E: int, H: int) -> float:
+    """Bound factor of a chunk router's fast logits (include/moe.h)."""
+    return float(lib().moe_router_gamma(T, E, H))

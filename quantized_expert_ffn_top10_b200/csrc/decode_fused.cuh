@@ -88,6 +88,8 @@ struct DecodeFusedArgs {
     double2* rec;            // [DF_NREP][T][E] (logit, error bound): CTA c reads copy c % DF_NREP
     uint16_t* hB;            // [P][I] bf16, MMA-fragment order within each 32-block
     unsigned int* bar;       // grid barrier counters and flag, DF_BAR_WORDS words (zeroed before launch)
+    unsigned spin_limit;     // polling bound of the grid barriers (MOE_SPIN_LIMIT; lowered only by a test)
+    unsigned bar1_extra;     // 0; a test sets it to make grid barrier 1 unsatisfiable
     DfPlan pl;
 };
 
@@ -166,12 +168,16 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
 // lines of `bar` (zeroed before launch) and only grow.  Bounded: on expiry the
 // status word gets MOE_ERR_TIMEOUT and every thread of the CTA sees false.
 #define DF_BAR_GROUPS 16
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned ph, int site) {
+// spin_limit bounds the polling (MOE_SPIN_LIMIT unless a test lowers it);
+// extra > 0 (a test setting) makes the barrier wait for arrivals that never
+// come, so that every waiter runs into that bound.
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned ph, int site, unsigned spin_limit,
+                                             unsigned extra = 0) {
     __syncthreads();
     int ok = 1;
     if (threadIdx.x == 0) {
         const unsigned G = gridDim.x, NG = min(G, (unsigned)DF_BAR_GROUPS), grp = blockIdx.x % NG;
-        const unsigned members = (G - grp + NG - 1) / NG;
+        const unsigned members = (G - grp + NG - 1) / NG + extra;
         unsigned* flag = bar + 32 * (DF_BAR_GROUPS + 1);
         __threadfence();
         if (atomicAdd(bar + 32 * grp, 1u) + 1u == ph * members &&
@@ -180,7 +186,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned ph, int sit
         } else {
             unsigned it = 0;
             while (ld_acquire_u32(flag) < ph) {
-                if (++it > MOE_SPIN_LIMIT) { moe_note_timeout(site, (int)(ld_acquire_u32(flag) % 1000)); ok = 0; break; }
+                if (++it > spin_limit) { moe_note_timeout(site, (int)(ld_acquire_u32(flag) % 1000)); ok = 0; break; }
                 if (it > 16) __nanosleep(32);
             }
         }
@@ -721,7 +727,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         for (int c = 0; c < DF_NREP; ++c) a.rec[((size_t)c * T + t) * E + e] = r;
     }
     {
-        const bool gb = grid_barrier(a.bar, 1u, 1);
+        const bool gb = grid_barrier(a.bar, 1u, 1, a.spin_limit, a.bar1_extra);
         alive = __syncthreads_and(alive && gb) != 0;  // uniform across the CTA
     }
 
@@ -925,7 +931,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         }
     }
     {
-        const bool gb = grid_barrier(a.bar, 2u, 2);
+        const bool gb = grid_barrier(a.bar, 2u, 2, a.spin_limit);
         alive = __syncthreads_and(cok && gb) != 0;
     }
 

@@ -69,6 +69,8 @@ std::atomic<uint64_t> g_launches{0};
 uint64_t g_init_mask[4] = {0, 0, 0, 0};  // devices whose kernel attributes are set
 int g_df_grid[256];                     // fused-decode grid (one CTA per SM) per device, 0 = unusable
 int g_df_maxdyn[256];                   // its dynamic shared-memory limit per device
+std::atomic<unsigned> g_dbg_spin{0};    // test setting: grid-barrier polling bound (0 = MOE_SPIN_LIMIT)
+std::atomic<unsigned> g_dbg_bar1{0};    // test setting: extra arrivals grid barrier 1 waits for
 constexpr int kDfMaxH = 2560;           // largest H the fused decode kernel stages
 
 inline void stage(int i, cudaStream_t st) {
@@ -403,6 +405,8 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     a.bar = reinterpret_cast<unsigned int*>(c.ws + L.gbar);
     a.rec = reinterpret_cast<double2*>(c.ws + L.rec);
     a.pl = plan;
+    a.spin_limit = g_dbg_spin.load() ? g_dbg_spin.load() : MOE_SPIN_LIMIT;
+    a.bar1_extra = g_dbg_bar1.load();
     CUtensorMap tm[2];
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
     if (!tmap_codes_gu(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8,
@@ -567,18 +571,44 @@ int moe_route(const uint16_t* x, int T, int H, const float* router_w, const floa
 static __device__ __align__(256) uint8_t g_route_scratch[MOE_ROUTE_STATIC_BYTES];
 
 namespace {
-void* g_route_scratch_addr[256];  // per device, filled on first use under g_mu
+// Per device: the address of g_route_scratch and the CUDA context it was
+// looked up in.  A different current context on the device (after
+// cudaDeviceReset, or a context the caller made current) has its own copy of
+// the array, so the address is looked up again there.
+void* g_route_scratch_addr[256];
+CUcontext g_route_scratch_ctx[256];
 
-// Address of this device's g_route_scratch, looked up once with the device current.
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    });
+    return fn;
+}
+
+// Address of g_route_scratch in the current context of the current device.
+// The first call in a context does the lookup (cudaGetSymbolAddress); later
+// calls in that context only compare the context handle.
 int route_scratch(uint8_t** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return MOE_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    PFN_cuCtxGetCurrent_v4000 get = ctx_getter();
+    if (!get || get(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> g(g_mu);
-    if (!g_route_scratch_addr[dev]) {
+    if (!ctx || !g_route_scratch_addr[dev] || g_route_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
+        // (also makes the device's primary context current when no context is)
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
         if (!aligned(p, kAlign)) return MOE_ERR_CUDA;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx) return MOE_ERR_CUDA;
         g_route_scratch_addr[dev] = p;
+        g_route_scratch_ctx[dev] = ctx;
     }
     *out = static_cast<uint8_t*>(g_route_scratch_addr[dev]);
     return MOE_OK;
@@ -676,6 +706,31 @@ int moe_set_stage_events(void* const* events, int n) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_debug_set(int key, int value) {
+    if (value < 0) return MOE_ERR_RANGE;
+    switch (key) {
+        case MOE_DBG_SPIN_LIMIT: g_dbg_spin = (unsigned)value; return MOE_OK;
+        case MOE_DBG_BARRIER_EXTRA: g_dbg_bar1 = (unsigned)value; return MOE_OK;
+        default: return MOE_ERR_ARG;
+    }
+}
+
+size_t moe_workspace_offset(int T, int E, int top_k, int H, int I, int field) {
+    if (T < 1 || E < 1 || top_k < 1 || H < 1 || I < 1) return (size_t)-1;
+    const Ws L = ws_layout(T, E, top_k, H, I);
+    switch (field) {
+        case MOE_WS_FAST_LOGITS: return L.logit;
+        case MOE_WS_PAIR_OUT: return L.y;
+        default: return (size_t)-1;
+    }
+}
+
+double moe_router_gamma(int T, int E, int H) {
+    if (T <= MOE_DECODE_MAX_T || E < 1 || E > MOE_MAX_E || H < 32 || H % 32) return -1.0;
+    if (E % RT_BM == 0 && H % RT_BK == 0) return moe_tc_router_gamma(H);  // tensor-core chunk router
+    return gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);      // CUDA-core chunk router
+}
 
 int moe_timeout_site(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;

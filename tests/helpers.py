@@ -16,6 +16,14 @@ import oracle as O
 
 OUT_RTOL = 2e-2
 W_ATOL = 1e-4
+# Per-pair expert outputs w * y of the prefill path are intermediates, not layer
+# outputs: the weights, h and the stored value are each rounded once to bf16
+# and there is no residual to dominate the row.  A CPU emulation of exactly
+# those roundings (tests/test_tolerance_model.py) reaches 2.1e-2 elementwise
+# (relative to max(|r|, row rms)) about once in 10^6 elements and 0.5e-2
+# normwise; the checks on them use 3e-2 elementwise and 1e-2 normwise.
+PAIR_RTOL = 3e-2
+PAIR_NORM_RTOL = 1e-2
 
 
 def bits_to_f32(bits: np.ndarray) -> np.ndarray:

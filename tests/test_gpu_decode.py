@@ -186,3 +186,36 @@ def test_fused_decode_repeated_calls_are_identical(decode_wl):
     o1, r1 = run_layer(decode_wl, 0, x, prefill=False)
     o2, r2 = run_layer(decode_wl, 0, x, prefill=False)
     assert np.array_equal(o1, o2) and np.array_equal(r1["perm"], r2["perm"])
+
+
+def test_fused_decode_wait_expiry_reports_timeout(cuda_ok):
+    """A bounded wait that runs out: with the test hooks, the fused kernel's
+    first grid barrier waits for an arrival that never comes and gives up
+    after a few thousand polls.  At that barrier no CTA has a copy in flight
+    or tensor memory allocated, so every CTA leaves cleanly; the call reports
+    MOE_ERR_TIMEOUT at site 1, and the next normal call is correct."""
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    cfg = S.config("tiny", E=16, top_k=4, H=1024, I=256, T=3, router_std=None, seed=24)
+    wl = Workload(cfg)
+    x = wl.x_host()
+    xt = torch.from_numpy(x.view(np.int16)).cuda()
+    out = torch.zeros_like(xt)
+    ws = torch.empty(M.moe_workspace_bytes(3, cfg.E, cfg.top_k, cfg.H, cfg.I), dtype=torch.uint8, device="cuda")
+    assert M.moe_last_device_error() == 0 and M.moe_timeout_site() == 0
+    n0 = M.moe_launch_count()
+    try:
+        M.moe_debug_set(M.MOE_DBG_SPIN_LIMIT, 2000)
+        M.moe_debug_set(M.MOE_DBG_BARRIER_EXTRA, 1)
+        M.moe_forward_decode(wl.desc, wl.arena, wl.slot_table, 1, 0, xt, wl.W[0], None, cfg.top_k, True, out,
+                             ws=ws)
+        torch.cuda.synchronize()
+    finally:
+        M.moe_debug_set(M.MOE_DBG_SPIN_LIMIT, 0)
+        M.moe_debug_set(M.MOE_DBG_BARRIER_EXTRA, 0)
+    assert M.moe_launch_count() - n0 == 1, "the fused kernel (not the multi-kernel path) must have run"
+    assert M.moe_last_device_error() == M.MOE_ERR_TIMEOUT
+    site = M.moe_timeout_site()
+    assert site // 1000000 == 1, f"timeout site {site}"
+    assert M.moe_last_device_error() == 0 and M.moe_timeout_site() == 0  # both read-and-clear
+    _compare(wl, 0, x)

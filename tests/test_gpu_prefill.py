@@ -4,7 +4,7 @@ import pytest
 
 import moe_synth as S
 import oracle as O
-from helpers import Workload, assert_out_close, check_routing, run_layer
+from helpers import PAIR_NORM_RTOL, PAIR_RTOL, Workload, assert_out_close, check_routing, run_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -95,7 +95,73 @@ def test_prefill_full_chunk_uniform(cuda_ok):
     assert counts.sum() == 8192 * 10
 
 
-def test_prefill_stack_layer_zipf(cuda_ok):
-    """One layer of the 48 x 512, 2/2/4-bit, Zipf-routed stack at full size."""
-    counts = _full_size(S.config("prefill_stack"), layer=7)
-    assert counts.max() > 1000 and counts.min() < 50
+def _pair_outputs(ws, cfg, T, sel):
+    """Rows `sel` (pair positions) of the per-pair expert outputs w * y (bf16)
+    the prefill call left in its workspace."""
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    off = M.moe_workspace_offset(T, cfg.E, cfg.top_k, cfg.H, cfg.I, M.MOE_WS_PAIR_OUT)
+    Y = ws[off:off + T * cfg.top_k * cfg.H * 2].view(torch.int16).view(T * cfg.top_k, cfg.H)
+    return Y[torch.from_numpy(np.asarray(sel, np.int64)).cuda()].cpu().numpy().view(np.uint16)
+
+
+def test_prefill_stack_48_layers_teacher_forced(cuda_ok):
+    """The 48 x 512, 2/2/4-bit, Zipf-routed stack at full size (T = 8,192),
+    the library chaining its own bf16 outputs layer to layer; at every layer the
+    oracle takes the library's input to that layer (teacher forcing) and checks:
+      - the routing of all 8,192 tokens (indices, offsets, permutation) bit-exact;
+      - the layer output of 64 sampled tokens;
+      - every routed pair of the 3 most- and the 3 least-loaded experts, on the
+        per-pair expert outputs w * y (bf16 intermediates: PAIR_RTOL);
+    and at the end the 48 x 512 histogram bit-exact and its ranking equal to the
+    oracle's."""
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    cfg = S.config("prefill_stack")
+    wl = Workload(cfg)
+    T, E, k = cfg.T, cfg.E, cfg.top_k
+    x = wl.x_host()
+    hist = torch.zeros((cfg.L, E), dtype=torch.int32, device="cuda")
+    ref_hist = np.zeros((cfg.L, E), np.uint32)
+    ws = torch.empty(M.moe_workspace_bytes(T, E, k, cfg.H, cfg.I), dtype=torch.uint8, device="cuda")
+    rng = np.random.default_rng(cfg.seed)
+    loads = []
+    for layer in range(cfg.L):
+        xt = torch.from_numpy(x.view(np.int16)).cuda()
+        out = torch.zeros_like(xt)
+        from helpers import route_buffers
+        ro = route_buffers(T, k, E)
+        M.moe_forward_prefill(wl.desc, wl.arena, wl.slot_table, cfg.L, layer, xt, wl.W[layer], wl.b[layer], k,
+                              True, out, hist=hist, route_out=ro, ws=ws)
+        torch.cuda.synchronize()
+        assert M.moe_last_device_error() == 0
+        res = {key: v.cpu().numpy() for key, v in ro.items()}
+        res["topk_idx"] = res["topk_idx"].reshape(T, k)
+        res["topk_w"] = res["topk_w"].reshape(T, k)
+        lg = O.router_logits(x, wl.W_host[layer], wl.b_host[layer])
+        idx, w = O.topk(lg, k)
+        counts = check_routing(res, idx, w, E)
+        O.hist_add(counts, layer, ref_hist)
+        loads.append((int(counts.max()), int(counts[counts > 0].min())))
+        ob = out.cpu().numpy().view(np.uint16)
+        toks = np.sort(rng.choice(T, 64, replace=False)).astype(np.int32)
+        ref = wl.oracle_layer(layer, x, tokens=toks)
+        assert_out_close(ob, ref["out_f64"], rows=toks)
+        # every pair of the 3 most- and 3 least-loaded (nonzero) experts
+        _, offsets, perm, _ = O.permutation(idx, E)
+        used = np.nonzero(counts)[0]
+        order = used[np.argsort(counts[used], kind="stable")]
+        xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        for e in list(order[:3]) + list(order[-3:]):
+            pos = np.arange(offsets[e], offsets[e + 1])
+            pairs = perm[pos]
+            s = int(wl.slot_table_host[layer * E + e])
+            y, _ = O.expert_ffn_rows(wl.slot_bytes_of(s), wl.desc, xf[pairs // k])
+            r = w.reshape(-1)[pairs][:, None] * y
+            rel = assert_out_close(_pair_outputs(ws, cfg, T, pos), r, tol=PAIR_RTOL)
+            assert rel <= PAIR_NORM_RTOL
+        x = ob
+    got = hist.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref_hist)
+    assert np.array_equal(M.moe_rank_experts(got), O.rank(ref_hist))
+    assert max(m for m, _ in loads) > 1000 and min(n for _, n in loads) < 50

@@ -320,3 +320,85 @@ def test_page_shapes_match_workloads():
     assert S.config("decode").T == 1 + facts["spec_drafts"]["value"]
     assert round(facts["vram_slots_12gb"]["value"] / facts["experts_total_pruned"]["value"], 2) == \
         facts["random_hit_rate"]["value"]
+
+
+# ------------------------------------------------------------------ pins added with the bulk expert check
+
+def test_router_two_term_hand_case():
+    """x = (1.5, -0.25) on two coordinates: l_e = 1.5 W[e, 3] - 0.25 W[e, 9] + b_e,
+    written out by hand for chosen exactly representable weights."""
+    E, H = 3, 16
+    W = np.zeros((E, H), np.float32)
+    W[0, 3], W[0, 9] = 2.0, 4.0          # 3 - 1 = 2
+    W[1, 3], W[1, 9] = -1.0, 0.5         # -1.5 - 0.125 = -1.625
+    W[2, 3], W[2, 9] = 0.125, -8.0       # 0.1875 + 2 = 2.1875
+    b = np.array([0.5, 0.0, -0.25], np.float32)
+    x = np.zeros((1, H), np.float32)
+    x[0, 3], x[0, 9] = 1.5, -0.25
+    lg = O.router_logits(_bf16(x), W, b)
+    assert lg[0].tolist() == [2.5, -1.625, 1.9375]
+    assert O.topk(lg, 2)[0].tolist() == [[0, 2]]
+
+
+def test_histogram_per_expert_hand_case():
+    """Counts land on their own (layer, expert) cell: a count moved to another
+    expert of the same layer keeps the per-layer total but fails here."""
+    hist = np.zeros((2, 4), np.uint32)
+    O.hist_add(np.array([3, 0, 1, 6], np.int32), 1, hist)
+    O.hist_add(np.array([0, 2, 0, 0], np.int32), 0, hist)
+    O.hist_add(np.array([1, 1, 1, 1], np.int32), 1, hist)
+    assert hist.tolist() == [[0, 2, 0, 0], [4, 1, 2, 7]]
+    idx = np.array([[2, 0], [2, 3], [3, 2]], np.int32)   # 3 tokens, k = 2, E = 4
+    counts, *_ = O.permutation(idx, 4)
+    assert counts.tolist() == [1, 0, 3, 2]
+
+
+def test_fp64_router_decides_a_tie_that_fp32_sums_lose():
+    """The oracle's logits are fp64 sums of exact products.  Two router rows
+    that differ by one fp32 ulp in one weight give fp64 logits that differ by
+    that product exactly, while fp32 sequential sums of the same products round
+    the difference away: the fp64 order (the higher index first here) is the
+    one the oracle - and the GPU, which certifies against it - reports."""
+    rng = np.random.default_rng(41)
+    H = 2048
+    x = _bf16(rng.standard_normal((1, H)).astype(np.float32))
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    W = np.zeros((2, H), np.float32)
+    W[0] = (rng.standard_normal(H) / np.sqrt(H)).astype(np.float32)
+    W[1] = W[0]
+    h = int(np.argmin(np.abs(xf[0])))                  # the smallest |x_h|: a tiny difference
+    if xf[0, h] == 0:
+        h = int(np.argsort(np.abs(xf[0]))[np.count_nonzero(xf[0] == 0)])
+    W[1, h] = np.nextafter(W[0, h], np.float32(np.inf) if xf[0, h] > 0 else np.float32(-np.inf))
+    lg = O.router_logits(x, W, None)
+    assert lg[0, 1] > lg[0, 0]                         # fp64: row 1 strictly ahead
+    assert lg[0, 1] - lg[0, 0] == pytest.approx(float(xf[0, h]) * (float(W[1, h]) - float(W[0, h])), rel=1e-6)
+    f32 = np.zeros(2, np.float32)
+    for e in range(2):                                  # fp32 sums in index order
+        s = np.float32(0)
+        for i in range(H):
+            s = np.float32(s + np.float32(xf[0, i] * W[e, i]))
+        f32[e] = s
+    assert f32[0] == f32[1]                             # fp32: an exact tie (row 0 would win)
+    assert O.topk(lg, 1)[0].tolist() == [[1]]
+
+
+def test_expert_ffn_rows_matches_per_element_oracle():
+    """The whole-matrix restatement against the per-element C oracle (itself
+    pinned above by closed forms) on random slots of each bit layout."""
+    rng = np.random.default_rng(42)
+    for bits in [(4, 4, 4), (2, 2, 4), (2, 4, 2)]:
+        cfg = S.config("tiny", H=128, I=64, bits=bits, seed=43)
+        d = cfg.desc()
+        slot = S.gen_slot_host(cfg, 3)
+        X = rng.standard_normal((5, cfg.H))
+        Y, Hh = O.expert_ffn_rows(slot, d, X)
+        for t in range(5):
+            y, h = O.expert_ffn(slot, d, X[t])
+            assert np.allclose(Y[t], y, rtol=1e-12, atol=1e-14)
+            assert np.allclose(Hh[t], h, rtol=1e-12, atol=1e-14)
+        for m in range(3):
+            rows, K = S.matrix_shape(cfg.H, cfg.I, m)
+            Wm = O.dequant_matrix(slot, d, m)
+            for r, c in [(0, 0), (rows - 1, K - 1), (rows // 2, 33), (1, K // 2 + 7)]:
+                assert Wm[r, c] == O.dequant(slot, d, m, r, c)

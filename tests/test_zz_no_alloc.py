@@ -70,3 +70,51 @@ def test_static_route_rejects_T_beyond_limit(cuda_ok):
     assert rc == M.MOE_ERR_STATIC
     torch.cuda.synchronize()
     assert int((ro["topk_idx"] != -1).sum()) == 0  # nothing was launched
+
+
+_FRESH = r"""
+import sys
+sys.path.insert(0, sys.argv[1])
+import numpy as np, torch
+import moe_synth as S
+import quantized_expert_ffn_top10_b200 as M
+cfg = S.config("decode_stack")
+T, k, E = 8, cfg.top_k, cfg.E
+outs = []
+for call in range(2):
+    x = torch.from_numpy(S.gen_x(cfg, T=T, stream_offset=call).view(np.int16)).cuda()
+    W = torch.from_numpy(S.gen_router(cfg)).cuda()
+    b = torch.from_numpy(S.gen_bias(cfg)).cuda()
+    res = []
+    for static in (True, False):  # the no-workspace call first: nothing else has run in this process
+        idx = torch.full((T * k,), -1, dtype=torch.int32, device="cuda")
+        w = torch.zeros(T * k, dtype=torch.float32, device="cuda")
+        off = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+        perm = torch.full((T * k,), -1, dtype=torch.int32, device="cuda")
+        if static:
+            M.moe_route_static(x, W, b, k, idx, w, off, perm)
+        else:
+            ws = torch.empty(M.moe_workspace_bytes(T, E, k, cfg.H, 32), dtype=torch.uint8, device="cuda")
+            M.moe_route(x, W, b, k, idx, w, off, perm, ws)
+        torch.cuda.synchronize()
+        assert M.moe_last_device_error() == 0
+        res.append([t.cpu().numpy() for t in (idx, w, off, perm)])
+    (i1, w1, o1, p1), (i2, w2, o2, p2) = res
+    assert np.array_equal(i1, i2) and np.array_equal(o1, o2) and np.array_equal(p1, p2)
+    assert np.max(np.abs(w1 - w2)) <= 1e-4
+print("fresh-process static route ok")
+"""
+
+
+@pytest.mark.gpu
+def test_static_route_in_a_fresh_process(cuda_ok):
+    """The same comparison in a new Python process whose first library call is
+    moe_route_static (T = 8, the limit), so that the scratch address lookup
+    runs with nothing initialised before it."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FRESH, root], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    assert "fresh-process static route ok" in r.stdout

@@ -161,15 +161,20 @@ int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, con
  * selected expert's weights are read once per window).
  *   desc (host); arena (device, 256-B aligned); slot_table [L][E] int32
  *   (device); x [T][H] bf16 (device); out [T][H] bf16 (device);
+ *   steer [H] fp32 (device, 16-B aligned) or NULL: the steering projection of
+ *   the "Coder benchmark record" page (steering vector section) - each output
+ *   row h (residual included) becomes h - (h . v) v before its one bf16
+ *   rounding, v = steer used as given (a unit vector is the caller's
+ *   business); NULL = no projection;
  *   hist [L][E] uint32 (device, persistent, caller-owned) or NULL;
  *   route_out (host struct of device pointers) or NULL.
  *   0 <= layer < L.  T = 0 is a no-op.
  */
 int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
                        int L, int layer, const uint16_t* x, int T, const float* router_w,
-                       const float* router_bias, int E, int top_k, int residual, uint16_t* out,
-                       uint32_t* hist, const moe_route_out* route_out, void* ws, size_t ws_bytes,
-                       void* stream);
+                       const float* router_bias, int E, int top_k, int residual, const float* steer,
+                       uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /*
  * Full layer for a prefill chunk, 1 <= T <= MOE_PREFILL_MAX_T: same arguments
@@ -183,9 +188,9 @@ int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int3
  */
 int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
                         int L, int layer, const uint16_t* x, int T, const float* router_w,
-                        const float* router_bias, int E, int top_k, int residual, uint16_t* out,
-                        uint32_t* hist, const moe_route_out* route_out, void* ws, size_t ws_bytes,
-                        void* stream);
+                        const float* router_bias, int E, int top_k, int residual, const float* steer,
+                        uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /*
  * Routing-count histogram ("--dump-routing" counts of the benchmark record
@@ -207,8 +212,42 @@ int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, 
  */
 int moe_rank_experts(const uint32_t* hist_host, int L, int E, uint16_t* pairs_out);
 
+/*
+ * Expert profile file in the STRP v1 layout of the "Coder benchmark record"
+ * page, "expert profile file": the magic "STRP", a header of five uint32
+ * (version = 1, layers L, experts per layer E, ranked pairs n, inverse-table
+ * entries = L*E), the n ranked (layer, expert) pairs as two uint16 each in
+ * rank order, then one inverse table per layer of E int32 entries giving the
+ * rank of (layer, expert), -1 = unranked (O(1) lookup of a pair's place).
+ * All fields little-endian.  The page lists the header fields without
+ * saying which of its two counts is which; here "ranked pairs" counts the
+ * body and "entries" the inverse tables.  Host only, no CUDA.
+ * moe_profile_bytes: the file size for (n_pairs, L, E), -1 if out of range
+ *   (1 <= L, E <= 65535, 0 <= n_pairs <= L*E).
+ * moe_profile_write: pairs [n_pairs][2] uint16 (host) = (layer, expert) in
+ *   rank order, e.g. a prefix of moe_rank_experts' output; writes the file
+ *   into buf (host, buf_bytes) and returns its size, or the size alone when
+ *   buf == NULL; MOE_ERR_ARG for a pair out of range or ranked twice,
+ *   MOE_ERR_WS when buf is too small, MOE_ERR_RANGE for bad sizes.
+ * moe_profile_read: parses and validates a file; fills L, E, n_pairs and,
+ *   when not NULL, pairs [n_pairs][2] and inverse [L*E]; MOE_ERR_SHAPE for a
+ *   malformed file.
+ * moe_profile_hit_rate: the slot-budget simulator of the same page ("why a
+ *   72% hit rate proves the mapping"): with the first `slots` ranked pairs
+ *   resident, the fraction of the routed reads counted in hist [L][E] (host,
+ *   e.g. a routing histogram of a held-out run) that land on a resident pair;
+ *   -1 on bad arguments.
+ */
+int64_t moe_profile_bytes(int n_pairs, int L, int E);
+int64_t moe_profile_write(const uint16_t* pairs, int n_pairs, int L, int E, uint8_t* buf, size_t buf_bytes);
+int moe_profile_read(const uint8_t* buf, size_t bytes, int* L, int* E, int* n_pairs, uint16_t* pairs,
+                     int32_t* inverse);
+double moe_profile_hit_rate(const uint16_t* pairs, int n_pairs, int L, int E, int slots, const uint32_t* hist);
+
 /* Reads and clears the current device's status word after synchronising
- * `stream`: MOE_OK, MOE_ERR_SLOT or MOE_ERR_TIMEOUT (the first latched). */
+ * `stream`: MOE_OK, MOE_ERR_SLOT or MOE_ERR_TIMEOUT (the first latched), or
+ * MOE_ERR_RANGE if an internal index was out of range and replaced (a
+ * library fault; inputs cannot cause it: non-finite logits rank as -inf). */
 int moe_last_device_error(void* stream);
 
 /* Static message for a return code. */
@@ -243,7 +282,9 @@ uint64_t moe_launch_count(void);
  *   or route workspace of MOE_WS_FAST_LOGITS (the router's fast logits: fp32
  *   [T][E] for chunks T > MOE_DECODE_MAX_T, fp64 for decode windows) or
  *   MOE_WS_PAIR_OUT (per-pair expert outputs w * y in pair order: bf16 [T*k][H]
- *   for chunks); (size_t)-1 for bad arguments.
+ *   for chunks) or MOE_WS_SLOW_COUNT (int32: how many tokens of a chunk the
+ *   fast certification could not decide, then their ids); (size_t)-1 for bad
+ *   arguments.
  * moe_router_gamma(T, E, H): for a chunk (T > MOE_DECODE_MAX_T), the factor
  *   gamma of the fast logits' certified bound |fast - exact| <= gamma *
  *   (||x_t|| ||W_r[e]|| + |b_e|) (before the fp64 definition's own rounding
@@ -253,6 +294,7 @@ uint64_t moe_launch_count(void);
 #define MOE_DBG_BARRIER_EXTRA 2
 #define MOE_WS_FAST_LOGITS 1
 #define MOE_WS_PAIR_OUT 2
+#define MOE_WS_SLOW_COUNT 3
 int moe_debug_set(int key, int value);
 size_t moe_workspace_offset(int T, int E, int top_k, int H, int I, int field);
 double moe_router_gamma(int T, int E, int H);

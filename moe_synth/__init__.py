@@ -129,23 +129,34 @@ class LayerConfig:
         return make_desc(self.H, self.I, self.bits, n_slots=self.L * self.E)
 
 
+# Expert scales of the two 48-layer stacks.  The layer is x + MoE(x) with no
+# normalisation, and a SwiGLU expert grows with |x|^2, so a chain of random
+# layers diverges unless the MoE part stays small: with the tiny workload's
+# U(0.001, 0.01) a token's residual stream overflows within about 10 layers.
+# U(0.0002, 0.002) keeps every token bounded over 48 layers.
+STACK_SCALE = (0.0002, 0.002)
+
+
 def config(name: str, **over) -> LayerConfig:
     """The named workloads.
 
     tiny        : L=1, E=8, k=2, H=64, I=32, T=4, router std 0.02, seed 0
     decode      : L=1, E=512, k=10, H=2048, I=512, T=5 (T=1 via override), seed 1
-    decode_stack: L=48, E=256, k=10, T=5, gate/up 2-bit, down 4-bit, Zipf 1.1, seed 2
+    decode_stack: L=48, E=256, k=10, T=5, gate/up 2-bit, down 4-bit, Zipf 1.1, seed 2,
+                  scales STACK_SCALE
     prefill     : L=1, E=512, k=10, T=8192, 4-bit, no bias, seed 3
-    prefill_stack: L=48, E=512, k=10, T=8192, 2/2/4-bit, Zipf 1.1, seed 4
+    prefill_stack: L=48, E=512, k=10, T=8192, 2/2/4-bit, Zipf 1.1, seed 4, scales STACK_SCALE
     """
     base = {
         "tiny": LayerConfig("tiny", 1, 8, 2, 64, 32, 4, router_std=0.02, seed=0),
         "decode": LayerConfig("decode", 1, 512, 10, 2048, 512, 5, seed=1),
         "decode_stack": LayerConfig("decode_stack", 48, 256, 10, 2048, 512, 5,
-                                    bits=(2, 2, 4), zipf_s=1.1, seed=2),
+                                    bits=(2, 2, 4), zipf_s=1.1, seed=2, scale_lo=STACK_SCALE[0],
+                                    scale_hi=STACK_SCALE[1]),
         "prefill": LayerConfig("prefill", 1, 512, 10, 2048, 512, 8192, seed=3),
         "prefill_stack": LayerConfig("prefill_stack", 48, 512, 10, 2048, 512, 8192,
-                                     bits=(2, 2, 4), zipf_s=1.1, seed=4),
+                                     bits=(2, 2, 4), zipf_s=1.1, seed=4, scale_lo=STACK_SCALE[0],
+                                     scale_hi=STACK_SCALE[1]),
     }[name]
     for k, v in over.items():
         setattr(base, k, v)

@@ -68,8 +68,10 @@ def lib():
         L.oracle_rank.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
         L.oracle_moe_layer.restype = ctypes.c_int
         L.oracle_moe_layer.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P,
-                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P,
                                        ctypes.c_int]
+        L.oracle_steer.restype = None
+        L.oracle_steer.argtypes = [P, P, ctypes.c_int]
         L.oracle_set_threads.restype = None
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_max_threads.restype = ctypes.c_int
@@ -219,10 +221,19 @@ def rank(hist: np.ndarray) -> np.ndarray:
 
 # --------------------------------------------------------------- layer
 
+def steer(h: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """h - (h . v) v for one row (fp64), the C oracle_steer."""
+    h = _c(h, np.float64).copy()
+    v = _c(v, np.float32)
+    lib().oracle_steer(_p(h), _p(v), h.shape[0])
+    return h
+
+
 def moe_layer(desc, arena: np.ndarray, slot_table: np.ndarray, L: int, layer: int,
               x_bits: np.ndarray, W: np.ndarray, b: np.ndarray | None, k: int,
-              residual: bool = True, tokens: np.ndarray | None = None):
-    """Run the layer for all tokens (or the listed ones).
+              residual: bool = True, tokens: np.ndarray | None = None, steer: np.ndarray | None = None):
+    """Run the layer for all tokens (or the listed ones); `steer` [H] fp32
+    removes that direction from every output row before its rounding.
 
     Returns dict(out=bf16 bits [T,H], out_f64=[T,H], idx=[T,k], w=[T,k], rc=int);
     rows of unlisted tokens are left zero."""
@@ -239,8 +250,9 @@ def moe_layer(desc, arena: np.ndarray, slot_table: np.ndarray, L: int, layer: in
     w = np.zeros((T, k), np.float64)
     tok = _c(tokens, np.int32)
     nt = 0 if tok is None else tok.shape[0]
+    sv = _c(steer, np.float32)
     rc = lib().oracle_moe_layer(ctypes.byref(desc), _p(arena), _p(slot_table), L, layer,
-                                _p(x_bits), T, _p(W), _p(b), E, k, int(bool(residual)),
+                                _p(x_bits), T, _p(W), _p(b), E, k, int(bool(residual)), _p(sv),
                                 _p(out), _p(out64), _p(idx), _p(w), _p(tok), nt)
     return {"out": out, "out_f64": out64, "idx": idx, "w": w, "rc": rc}
 

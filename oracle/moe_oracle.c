@@ -174,6 +174,11 @@ void oracle_router_logits(const uint16_t* x, int T, int H, const float* W, const
     }
 }
 
+/* A logit as it takes part in the selection and the weights: NaN counts as
+ * -infinity (the pages fix nothing for non-finite values; this makes the order
+ * total, so a NaN logit ranks below every number and, if selected, weighs 0). */
+static double orc_ord(double v) { return isnan(v) ? -INFINITY : v; }
+
 /* Top-k by repeated selection: the j-th pick is the largest logit not yet
  * chosen, the lower expert index winning an exact tie.  Weights are the
  * softmax of the k chosen logits: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0). */
@@ -186,14 +191,14 @@ void oracle_topk(const double* logits, int T, int E, int k, int32_t* idx, double
             int best = -1;
             for (int e = 0; e < E; e++) {
                 if (taken[e]) continue;
-                if (best < 0 || l[e] > l[best]) best = e;   /* strict '>' keeps the lower index */
+                if (best < 0 || orc_ord(l[e]) > orc_ord(l[best])) best = e;   /* strict '>' keeps the lower index */
             }
             taken[best] = 1;
             idx[(int64_t)t * k + j] = best;
         }
-        double l0 = l[idx[(int64_t)t * k]], z = 0.0;
-        for (int j = 0; j < k; j++) z += exp(l[idx[(int64_t)t * k + j]] - l0);
-        for (int j = 0; j < k; j++) w[(int64_t)t * k + j] = exp(l[idx[(int64_t)t * k + j]] - l0) / z;
+        double l0 = orc_ord(l[idx[(int64_t)t * k]]), z = 0.0;
+        for (int j = 0; j < k; j++) z += exp(orc_ord(l[idx[(int64_t)t * k + j]]) - l0);
+        for (int j = 0; j < k; j++) w[(int64_t)t * k + j] = exp(orc_ord(l[idx[(int64_t)t * k + j]]) - l0) / z;
     }
     free(taken);
 }
@@ -253,9 +258,22 @@ void oracle_rank(const uint32_t* hist, int L, int E, uint16_t* pairs) {
 
 /* ---------------------------------------------------------------- layer */
 
+/* Steering projection of the "Coder benchmark record" page, section on the
+ * steering vector: after the layer, the component of the residual stream h
+ * along a unit direction v is removed, h - (h . v) v.  The dot product is
+ * summed in index order in fp64; v is used as given (its unit length is the
+ * caller's).  h has H entries and is updated in place. */
+void oracle_steer(double* h, const float* v, int H) {
+    double dot = 0.0;
+    for (int c = 0; c < H; c++) dot += h[c] * (double)v[c];
+    for (int c = 0; c < H; c++) h[c] -= dot * (double)v[c];
+}
+
 /* One MoE layer for the tokens listed in `tokens` (all T when tokens == NULL).
  *  x        [T][H] bf16 bits          W [E][H] fp32, b [E] fp32 or NULL
  *  arena    n_slots * slot_bytes       slot_table [L][E] int32
+ *  steer    [H] fp32 unit direction removed from each output row before its
+ *           rounding (oracle_steer), or NULL
  *  out      [T][H] bf16 bits (rows of listed tokens written)
  *  out_f64  [T][H] fp64 before rounding, optional
  *  idx, w   [T][k] routing of the listed tokens, optional
@@ -263,7 +281,7 @@ void oracle_rank(const uint32_t* hist, int L, int E, uint16_t* pairs) {
  * contributes 0), ORC_ERR_ARG on bad arguments, else ORC_OK. */
 int oracle_moe_layer(const orc_desc* d, const uint8_t* arena, const int32_t* slot_table,
                      int L, int layer, const uint16_t* x, int T, const float* W, const float* b,
-                     int E, int k, int residual, uint16_t* out, double* out_f64,
+                     int E, int k, int residual, const float* steer, uint16_t* out, double* out_f64,
                      int32_t* idx_out, double* w_out, const int32_t* tokens, int n_tokens) {
     if (!d || !arena || !slot_table || !x || !W || !out) return ORC_ERR_ARG;
     if (layer < 0 || layer >= L || k < 1 || k > E || T < 0) return ORC_ERR_ARG;
@@ -299,19 +317,23 @@ int oracle_moe_layer(const orc_desc* d, const uint8_t* arena, const int32_t* slo
         oracle_expert_ffn(arena + (int64_t)s * d->slot_bytes, d, xd, yp, NULL);
         free(xd);
     }
+    double* row = (double*)malloc(sizeof(double) * H);
     for (int i = 0; i < nt; i++) {
         int t = tokens ? tokens[i] : i;
         for (int c = 0; c < H; c++) {
             double acc = 0.0;
             for (int j = 0; j < k; j++) acc += w[(int64_t)i * k + j] * y[((int64_t)i * k + j) * H + c];
-            double v = residual ? oracle_bf16_to_double(xs[(int64_t)i * H + c]) + acc : acc;
-            if (out_f64) out_f64[(int64_t)t * H + c] = v;
-            out[(int64_t)t * H + c] = oracle_double_to_bf16(v);
+            row[c] = residual ? oracle_bf16_to_double(xs[(int64_t)i * H + c]) + acc : acc;
+        }
+        if (steer) oracle_steer(row, steer, H);
+        for (int c = 0; c < H; c++) {
+            if (out_f64) out_f64[(int64_t)t * H + c] = row[c];
+            out[(int64_t)t * H + c] = oracle_double_to_bf16(row[c]);
         }
         if (idx_out) memcpy(idx_out + (int64_t)t * k, idx + (int64_t)i * k, sizeof(int32_t) * k);
         if (w_out) memcpy(w_out + (int64_t)t * k, w + (int64_t)i * k, sizeof(double) * k);
     }
-    free(logit); free(xs); free(idx); free(w); free(y);
+    free(logit); free(xs); free(idx); free(w); free(y); free(row);
     return bad_slot ? ORC_ERR_SLOT : ORC_OK;
 }
 

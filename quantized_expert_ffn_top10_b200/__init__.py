@@ -45,9 +45,10 @@ MOE_ROUTE_STATIC_MAX_T, MOE_ROUTE_STATIC_BYTES = 8, 128 * 1024
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",
            "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
            "moe_set_stage_events", "moe_launch_count", "moe_timeout_site", "moe_route_static",
-           "moe_debug_set", "moe_workspace_offset", "moe_router_gamma")
+           "moe_debug_set", "moe_workspace_offset", "moe_router_gamma", "moe_profile_bytes",
+           "moe_profile_write", "moe_profile_read", "moe_profile_hit_rate")
 MOE_DBG_SPIN_LIMIT, MOE_DBG_BARRIER_EXTRA = 1, 2
-MOE_WS_FAST_LOGITS, MOE_WS_PAIR_OUT = 1, 2
+MOE_WS_FAST_LOGITS, MOE_WS_PAIR_OUT, MOE_WS_SLOW_COUNT = 1, 2, 3
 
 
 class RouteOut(ctypes.Structure):
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.moe_route.restype = i32
         L.moe_route.argtypes = [P, i32, i32, P, P, i32, i32, P, P, P, P, P, sz, P]
-        fwd = [P, P, P, i32, i32, P, i32, P, P, i32, i32, i32, P, P, P, P, sz, P]
+        fwd = [P, P, P, i32, i32, P, i32, P, P, i32, i32, i32, P, P, P, P, P, sz, P]
         L.moe_forward_decode.restype = i32
         L.moe_forward_decode.argtypes = fwd
         L.moe_forward_prefill.restype = i32
@@ -103,6 +104,14 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_offset.argtypes = [i32, i32, i32, i32, i32, i32]
         L.moe_router_gamma.restype = ctypes.c_double
         L.moe_router_gamma.argtypes = [i32, i32, i32]
+        L.moe_profile_bytes.restype = ctypes.c_int64
+        L.moe_profile_bytes.argtypes = [i32, i32, i32]
+        L.moe_profile_write.restype = ctypes.c_int64
+        L.moe_profile_write.argtypes = [P, i32, i32, i32, P, sz]
+        L.moe_profile_read.restype = i32
+        L.moe_profile_read.argtypes = [P, sz, P, P, P, P, P]
+        L.moe_profile_hit_rate.restype = ctypes.c_double
+        L.moe_profile_hit_rate.argtypes = [P, i32, i32, i32, i32, P]
         _lib = L
     return _lib
 
@@ -159,7 +168,7 @@ def moe_route_static(x, router_w, router_bias, top_k, topk_idx, topk_w, expert_o
 
 
 def _forward(fn, name, desc, arena, slot_table, L, layer, x, router_w, router_bias, top_k, residual, out,
-             hist, route_out, ws, stream, raise_on_error, T=None, E=None):
+             hist, route_out, ws, stream, raise_on_error, steer=None, T=None, E=None):
     T = x.shape[0] if T is None else T
     E = router_w.shape[0] if E is None else E
     ro = None
@@ -167,25 +176,30 @@ def _forward(fn, name, desc, arena, slot_table, L, layer, x, router_w, router_bi
         ro = RouteOut(*[_ptr(route_out.get(k)) for k in ("topk_idx", "topk_w", "expert_offsets", "perm",
                                                           "n_rechecked")])
     rc = fn(ctypes.byref(as_desc(desc)), _ptr(arena), _ptr(slot_table), L, layer, _ptr(x), T, _ptr(router_w),
-            _ptr(router_bias), E, top_k, int(bool(residual)), _ptr(out), _ptr(hist),
+            _ptr(router_bias), E, top_k, int(bool(residual)), _ptr(steer), _ptr(out), _ptr(hist),
             ctypes.byref(ro) if ro is not None else None, _ptr(ws),
             ws.numel() * ws.element_size() if hasattr(ws, "numel") else 0, _stream(stream))
     return _check(rc, name, raise_on_error)
 
 
 def moe_forward_decode(desc: ArenaDesc, arena, slot_table, L, layer, x, router_w, router_bias, top_k,
-                       residual, out, hist=None, route_out=None, ws=None, stream=None, raise_on_error=True):
+                       residual, out, hist=None, route_out=None, ws=None, stream=None, raise_on_error=True,
+                       steer=None):
     """One MoE layer for a decode window (T <= 8).  route_out: optional dict of
-    device tensors topk_idx / topk_w / expert_offsets / perm / n_rechecked."""
+    device tensors topk_idx / topk_w / expert_offsets / perm / n_rechecked;
+    steer: optional fp32 [H] direction projected out of every output row."""
     return _forward(lib().moe_forward_decode, "moe_forward_decode", desc, arena, slot_table, L, layer, x,
-                    router_w, router_bias, top_k, residual, out, hist, route_out, ws, stream, raise_on_error)
+                    router_w, router_bias, top_k, residual, out, hist, route_out, ws, stream, raise_on_error,
+                    steer=steer)
 
 
 def moe_forward_prefill(desc: ArenaDesc, arena, slot_table, L, layer, x, router_w, router_bias, top_k,
-                        residual, out, hist=None, route_out=None, ws=None, stream=None, raise_on_error=True):
+                        residual, out, hist=None, route_out=None, ws=None, stream=None, raise_on_error=True,
+                        steer=None):
     """One MoE layer for a prefill chunk (T <= 8192), tensor-core grouped GEMMs."""
     return _forward(lib().moe_forward_prefill, "moe_forward_prefill", desc, arena, slot_table, L, layer, x,
-                    router_w, router_bias, top_k, residual, out, hist, route_out, ws, stream, raise_on_error)
+                    router_w, router_bias, top_k, residual, out, hist, route_out, ws, stream, raise_on_error,
+                    steer=steer)
 
 
 def moe_route_histogram(expert_offsets, E, L, layer, hist, stream=None, raise_on_error=True) -> int:
@@ -243,3 +257,50 @@ def moe_workspace_offset(T: int, E: int, top_k: int, H: int, I: int, field: int)
 def moe_router_gamma(T: int, E: int, H: int) -> float:
     """Bound factor of a chunk router's fast logits (include/moe.h)."""
     return float(lib().moe_router_gamma(T, E, H))
+
+
+def moe_profile_write(pairs, L: int, E: int) -> bytes:
+    """STRP v1 expert profile (include/moe.h) of the ranked (layer, expert)
+    pairs (numpy uint16 [n, 2], rank order)."""
+    import numpy as np
+    pr = np.ascontiguousarray(pairs, dtype=np.uint16).reshape(-1, 2)
+    n = pr.shape[0]
+    size = int(lib().moe_profile_bytes(n, L, E))
+    if size < 0:
+        raise MoeError(MOE_ERR_RANGE, "moe_profile_bytes")
+    buf = np.zeros(size, np.uint8)
+    rc = int(lib().moe_profile_write(pr.ctypes.data_as(ctypes.c_void_p), n, L, E,
+                                     buf.ctypes.data_as(ctypes.c_void_p), size))
+    if rc < 0:
+        raise MoeError(rc, "moe_profile_write")
+    return buf.tobytes()
+
+
+def moe_profile_read(data: bytes):
+    """(L, E, pairs uint16 [n, 2], inverse int32 [L, E]) of an STRP v1 file."""
+    import numpy as np
+    raw = np.frombuffer(data, np.uint8).copy()
+    Lc, Ec, nc = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    P = ctypes.c_void_p
+    rc = lib().moe_profile_read(raw.ctypes.data_as(P), raw.size, ctypes.byref(Lc), ctypes.byref(Ec),
+                                ctypes.byref(nc), None, None)
+    _check(rc, "moe_profile_read", True)
+    pairs = np.zeros((nc.value, 2), np.uint16)
+    inv = np.zeros((Lc.value, Ec.value), np.int32)
+    rc = lib().moe_profile_read(raw.ctypes.data_as(P), raw.size, ctypes.byref(Lc), ctypes.byref(Ec),
+                                ctypes.byref(nc), pairs.ctypes.data_as(P), inv.ctypes.data_as(P))
+    _check(rc, "moe_profile_read", True)
+    return Lc.value, Ec.value, pairs, inv
+
+
+def moe_profile_hit_rate(pairs, L: int, E: int, slots: int, hist) -> float:
+    """Fraction of the routed reads in hist [L, E] that land in the first
+    `slots` ranked pairs."""
+    import numpy as np
+    pr = np.ascontiguousarray(pairs, dtype=np.uint16).reshape(-1, 2)
+    h = np.ascontiguousarray(hist, dtype=np.uint32)
+    v = float(lib().moe_profile_hit_rate(pr.ctypes.data_as(ctypes.c_void_p), pr.shape[0], L, E, slots,
+                                         h.ctypes.data_as(ctypes.c_void_p)))
+    if v < 0:
+        raise MoeError(MOE_ERR_ARG, "moe_profile_hit_rate")
+    return v

@@ -261,3 +261,56 @@ __global__ void __launch_bounds__(128) k_combine_bf16x8(const uint16_t* __restri
     o.w = (uint32_t)f32_to_bf16_bits(acc[6]) | ((uint32_t)f32_to_bf16_bits(acc[7]) << 16);
     *reinterpret_cast<uint4*>(out + (size_t)t * H + c) = o;
 }
+
+// ---------------------------------------------------------------- steering projection
+
+// The steering projection of the "Coder benchmark record" page (steering
+// vector section): the layer's output row h (residual included, fp32) loses
+// its component along the unit direction v, out = bf16(h - (h . v) v), with v
+// used as given.  One block per token.  h is either summed here from the
+// per-pair outputs y (fp32 or bf16, in slot order, then + x, as the plain
+// combine does) or read from hsrc; the dot product is summed in a fixed order
+// (each thread over its features in order, a fixed shuffle tree, the warps in
+// order), so repeated calls are bit-identical.
+#define STEER_THREADS 256
+
+template <typename YT>
+__global__ void __launch_bounds__(STEER_THREADS)
+    k_combine_steer(const uint16_t* __restrict__ x, const YT* __restrict__ y, const int32_t* __restrict__ inv,
+                    const float* __restrict__ hsrc, int T, int H, int k, int residual, const float* __restrict__ v,
+                    uint16_t* __restrict__ out) {
+    extern __shared__ float s_h[];  // [H]
+    __shared__ float s_red[STEER_THREADS / 32 + 1];
+    const int t = blockIdx.x;
+    if (t >= T) return;
+    float part = 0.f;
+    for (int c = threadIdx.x; c < H; c += STEER_THREADS) {
+        float h;
+        if (hsrc) {
+            h = hsrc[(size_t)t * H + c];
+        } else {
+            float acc = 0.f;
+            for (int j = 0; j < k; ++j) {
+                const size_t i = (size_t)inv[(size_t)t * k + j] * H + c;
+                if constexpr (sizeof(YT) == 4) acc += (float)y[i];
+                else acc += bf16_bits_to_f32((uint16_t)y[i]);
+            }
+            h = residual ? acc + bf16_bits_to_f32(x[(size_t)t * H + c]) : acc;
+        }
+        s_h[c] = h;
+        part = fmaf(h, v[c], part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float d = 0.f;
+        for (int w = 0; w < STEER_THREADS / 32; ++w) d += s_red[w];
+        s_red[STEER_THREADS / 32] = d;
+    }
+    __syncthreads();
+    const float dot = s_red[STEER_THREADS / 32];
+    for (int c = threadIdx.x; c < H; c += STEER_THREADS)
+        out[(size_t)t * H + c] = f32_to_bf16_bits(fmaf(-dot, v[c], s_h[c]));
+}

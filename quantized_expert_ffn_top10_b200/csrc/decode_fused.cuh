@@ -38,6 +38,25 @@
 #include "perm.cuh"
 #include "router.cuh"
 
+// Phase timestamps for measurement builds (-DMOE_PROBE): thread 0 of every
+// CTA records the global timer at the phase boundaries.  Compiled out
+// otherwise.
+#ifdef MOE_PROBE
+__device__ unsigned long long g_df_probe[160][16];
+#define DF_MARK(i)                                                                  \
+    do {                                                                            \
+        if (threadIdx.x == 0 && blockIdx.x < 160) {                                 \
+            unsigned long long t_;                                                  \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                  \
+            g_df_probe[blockIdx.x][i] = t_;                                         \
+        }                                                                           \
+    } while (0)
+#else
+#define DF_MARK(i) \
+    do {           \
+    } while (0)
+#endif
+
 #define DF_WARPS 16
 #define DF_THREADS (32 * DF_WARPS)
 #define DF_NBUF 2          // TMA slots per warp
@@ -72,11 +91,14 @@ struct DecodeFusedArgs {
     int64_t off_codes[3], off_scales[3];
     int64_t slot_bytes;
     int H, I, E, k, layer, T, residual;
+    int bits_gate, bits_up, bits_down;
     int epc;                 // router experts per CTA
     const uint16_t* x;       // [T][H]
     const float* W;          // router [E][H]
     const float* b;          // router bias [E] or null
     uint16_t* out;           // [T][H]
+    float* hout;             // [T][H] fp32 output rows before rounding (steering: a second kernel
+                             // finishes them), or null: bf16 rows go straight to out
     uint32_t* hist;          // [L][E] or null
     int32_t* idx;            // [T*k]
     float* w;                // [T*k]
@@ -120,7 +142,7 @@ __host__ inline bool df_plan(DfPlan& p, int T, int P, int E, int H, int I, int b
     // phase C
     const int xb = NB * 4 * T * 16;
     p.xc_off = o + xb;
-    p.part_off = p.xc_off + NB * DF_TN * 4;
+    p.part_off = p.xc_off + NB * 4 * 16;  // C quads [H/32][4]
     p.part_bytes = 2 * 16 * T * 4;
     p.n_part = df_max_tiles(P, E, I, G) + DF_WARPS;
     const int c_end = p.part_off + p.n_part * p.part_bytes;
@@ -213,13 +235,23 @@ __device__ __forceinline__ void unpack8(uint32_t w, uint32_t (&p)[4]) {
     }
 }
 
-// D(4 fp32) += A(16x16 bf16) * B(16x8 bf16)
+// D(4 fp32) += A(16x16 bf16) * B(16x8 bf16).  (Not volatile: a pure function
+// of its operands, which the compiler may schedule freely.)
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D(4 fp32) = A(16x16 bf16) * B(16x8 bf16) + C, with C a separate register
+// quad (loaded as one 16-byte value, so no copies into D are needed).
+__device__ __forceinline__ void mma_bf16_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1, const float4& c) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c.x), "f"(c.y), "f"(c.z), "f"(c.w));
 }
 
 // Byte offset, inside a 16-row box of 128-byte rows written with the TMA
@@ -345,8 +377,8 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
         const int e = lane + 32 * i;
         double2 r = make_double2(-INFINITY, 0.0);
         if (e < E) r = __ldcg(rec + e);
-        v[i] = r.x;
-        dl[i] = r.y;
+        v[i] = order_val(r.x);
+        dl[i] = order_bnd(r.y);
     }
     const int M = min(min(E, k + MOE_CAND_EXTRA), 32);
     double m = -INFINITY;
@@ -367,7 +399,7 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
         const bool valid = lane + 32 * i < E;
         const bool in = valid && v[i] >= th;
         bm[i] = __ballot_sync(0xffffffffu, in);
-        if (valid && !in) rest = fmax(rest, v[i] + dl[i]);
+        if (valid && !in) rest = fmax(rest, hi_end(v[i], dl[i]));
     }
     int nc = 0;
 #pragma unroll
@@ -415,8 +447,8 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
         const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
         const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
         bool ok = true;
-        if (lane < k && lane + 1 < nc) ok = (cval - cbnd) > (nv + nb);
-        if (lane == k - 1) ok = ok && (rest == -INFINITY || (cval - cbnd) > rest);
+        if (lane < k && lane + 1 < nc) ok = lo_end(cval, cbnd) > hi_end(nv, nb);
+        if (lane == k - 1) ok = ok && (rest == -INFINITY || lo_end(cval, cbnd) > rest);
         if (__all_sync(0xffffffffu, ok)) {
             write_topk(k, cval, ce, idx_out, w_out);
             return;
@@ -424,6 +456,17 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
     }
     __syncwarp();
     topk_token<2>(a, t, idx_out, w_out, cs, cvs, nrechk);
+}
+
+// ---------------------------------------------------------------- L2 prefetch of a selected expert
+
+// This CTA's 1/G slice [lo, lo + n) of expert slot `sl`, prefetched into L2.
+// Every CTA issues its slice of each selected expert as soon as a token's
+// selection is known, so the window's expert bytes start streaming from HBM
+// before the grouping is built and the first unit is requested; the units'
+// own loads then find them in L2 (or already in flight).
+__device__ __forceinline__ void df_prefetch_slot(const DecodeFusedArgs& a, int sl, uint32_t lo, uint32_t n) {
+    if (n > 0) prefetch_l2(a.arena + (int64_t)sl * a.slot_bytes + lo, n);
 }
 
 // ---------------------------------------------------------------- phase C: one gate/up unit
@@ -476,10 +519,10 @@ __device__ __forceinline__ float df_scale(const uint4* s, int j) {
 }
 
 // accg / accu (rows g, g + 8; token columns 2q, 2q + 1) += the unit's blocks
-// J0 .. J0 + NB - 1.  xb: x fragments [H/32][4][T]; xc: -(128 + offset) sum x
-// per (block, column) [H/32][8].
+// J0 .. J0 + NB - 1.  xb: x fragments [H/32][4][T]; xc: per (block, lane q)
+// the MMA's C quad (c_2q, c_2q+1, c_2q, c_2q+1), c = -(128 + offset) sum x.
 template <int BITS>
-__device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4* xb, const float* xc, int J0, int T,
+__device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4* xb, const float4* xc, int J0, int T,
                                              float (&accg)[4], float (&accu)[4]) {
     constexpr int NB = DfCRegs<BITS>::NB;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
@@ -488,7 +531,7 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
         const int J = J0 + j;
         uint4 bx = make_uint4(0u, 0u, 0u, 0u);
         if (g < T) bx = xb[(J * 4 + q) * T + g];
-        const float2 c = *reinterpret_cast<const float2*>(xc + J * DF_TN + 2 * q);
+        const float4 c = xc[J * 4 + q];
         const int sh = BITS == 2 ? 16 * (j & 1) : 0;
         const int wi = BITS == 2 ? (j >> 1) : j;
         uint32_t pg0[4], pg1[4], pu0[4], pu1[4];
@@ -496,10 +539,10 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
         unpack8<BITS>(r.g1[wi] >> sh, pg1);
         unpack8<BITS>(r.u0[wi] >> sh, pu0);
         unpack8<BITS>(r.u1[wi] >> sh, pu1);
-        float dg[4] = {c.x, c.y, c.x, c.y}, du[4] = {c.x, c.y, c.x, c.y};
-        mma_bf16_16816(dg, pg0[0], pg1[0], pg0[1], pg1[1], bx.x, bx.y);
+        float dg[4], du[4];
+        mma_bf16_16816_c(dg, pg0[0], pg1[0], pg0[1], pg1[1], bx.x, bx.y, c);
+        mma_bf16_16816_c(du, pu0[0], pu1[0], pu0[1], pu1[1], bx.x, bx.y, c);
         mma_bf16_16816(dg, pg0[2], pg1[2], pg0[3], pg1[3], bx.z, bx.w);
-        mma_bf16_16816(du, pu0[0], pu1[0], pu0[1], pu1[1], bx.x, bx.y);
         mma_bf16_16816(du, pu0[2], pu1[2], pu0[3], pu1[3], bx.z, bx.w);
         const float sg0 = df_scale(r.sg0, j), sg1 = df_scale(r.sg1, j);
         const float su0 = df_scale(r.su0, j), su1 = df_scale(r.su1, j);
@@ -586,7 +629,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     uint8_t* ring = base;               // code slots [warp][DF_NBUF][DF_CODE_SLOT]
     uint8_t* scr = base + pl.sc_off;    // scale slots [warp][DF_NBUF][sc_slot]
     uint4* xb = reinterpret_cast<uint4*>(base + pl.r1_off);
-    float* xc = reinterpret_cast<float*>(base + pl.xc_off);
+    float4* xc = reinterpret_cast<float4*>(base + pl.xc_off);
     float* part = reinterpret_cast<float*>(base + pl.part_off);
     DfRoute rt;
     rt.idx = reinterpret_cast<int32_t*>(base + pl.route_off);
@@ -616,6 +659,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    DF_MARK(0);
 
     // ---- A: router logits in fp64 on the tensor cores.  This CTA takes experts
     // e0 .. e0 + epc - 1 (rows of mma.m8n8k4.f64); its warps split H.  Every
@@ -635,6 +679,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         bulk_load(base + pl.stab_off, a.slot_table + (size_t)a.layer * E, (uint32_t)(E * 4), abar);
     }
     bool alive = mbar_wait(abar, 0, 1, 0);  // the x fragments are built while W_r is still arriving
+    DF_MARK(1);
     // x as MMA B fragments [H/32][4][T], its block sums and squares
     float* xp = reinterpret_cast<float*>(ring + pl.a_xp_off);  // [2][H/32][4][T]
     const int nxf = NB * 4 * T;
@@ -654,6 +699,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         xp[nxf + u] = sq;
     }
     alive = mbar_wait(wbar, 0, 1, 1) && alive;
+    DF_MARK(2);
     if (ne > 0) {
         const int g = lane >> 2, q = lane & 3;
         const int kw = H / DF_WARPS, kb = warp * kw;
@@ -700,14 +746,20 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         s_wn[lane] = sqrtf(s2) * 1.001f;
         a.wnorm[e0 + lane] = s_wn[lane];
     }
-    for (int u = tid; u < NB * DF_TN; u += DF_THREADS) {  // block corrections, zero beyond T
-        const int n = u % DF_TN, j = u / DF_TN;
-        float sx = 0.f;
-        if (n < T) {
-            const float* pp = xp + (size_t)j * 4 * T + n;
-            sx = ((pp[0] + pp[T]) + pp[2 * T]) + pp[3 * T];
+    for (int u = tid; u < NB * 4; u += DF_THREADS) {  // block corrections as MMA C quads, zero beyond T
+        const int q = u % 4, j = u / 4;
+        float sx[2];
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int n = 2 * q + z;
+            sx[z] = 0.f;
+            if (n < T) {
+                const float* pp = xp + (size_t)j * 4 * T + n;
+                sx[z] = ((pp[0] + pp[T]) + pp[2 * T]) + pp[3 * T];
+            }
         }
-        xc[u] = -(128.f + (float)(1 << (BGU - 1))) * sx;
+        const float f = -(128.f + (float)(1 << (BGU - 1)));
+        xc[u] = make_float4(f * sx[0], f * sx[1], f * sx[0], f * sx[1]);
     }
     __syncthreads();
     if (tid < 64 && (tid >> 3) < ne && (tid & 7) < T) {  // logits and their error bounds
@@ -726,12 +778,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < DF_NREP; ++c) a.rec[((size_t)c * T + t) * E + e] = r;
     }
+    DF_MARK(3);
     {
         const bool gb = grid_barrier(a.bar, 1u, 1, a.spin_limit, a.bar1_extra);
         alive = __syncthreads_and(alive && gb) != 0;  // uniform across the CTA
     }
+    DF_MARK(4);
 
     // ---- B: certified top-k of every token (same result in every CTA) and grouping
+    const uint32_t pf_step = (uint32_t)((a.slot_bytes / G + 15) & ~(int64_t)15);
+    const uint32_t pf_lo = pf_step * (uint32_t)cta;
+    const uint32_t pf_n = pf_lo >= a.slot_bytes ? 0u : (uint32_t)min((int64_t)pf_step, a.slot_bytes - pf_lo);
     if (alive) {
         if (warp < T) {
             TopkArgs ta{};
@@ -743,12 +800,27 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             double* cvs = reinterpret_cast<double*>(ring + warp * MOE_MAX_E * 12 + MOE_MAX_E * 4);
             const double2* rec = a.rec + ((size_t)(cta % DF_NREP) * T + warp) * E;
             df_topk_token(ta, rec, warp, rt.idx + warp * k, rt.w + warp * k, cs, cvs, cta == 0 ? a.nrechk : nullptr);
+            __syncwarp();
+            if (lane < k) {  // this token's experts start streaming into L2
+                const int e = rt.idx[warp * k + lane];
+                const int64_t sl = (unsigned)e < (unsigned)E ? stab[e] : -1;
+                if (sl >= 0 && sl < a.n_slots) df_prefetch_slot(a, (int)sl, pf_lo, pf_n);
+            }
         }
         int* s_cnt = reinterpret_cast<int*>(ring + pl.b_cnt_off);
         int* s_off = reinterpret_cast<int*>(ring + pl.b_off_off);
         for (int e = tid; e < MOE_MAX_E; e += DF_THREADS) s_cnt[e] = 0;
         __syncthreads();
-        for (int p = tid; p < P; p += DF_THREADS) atomicAdd(&s_cnt[rt.idx[p]], 1);
+        DF_MARK(5);
+        for (int p = tid; p < P; p += DF_THREADS) {
+            int e = rt.idx[p];
+            if ((unsigned)e >= (unsigned)E) {  // never produced by the top-k; a guard against a library fault
+                e = 0;
+                rt.idx[p] = 0;
+                moe_set_status(MOE_ERR_RANGE);
+            }
+            atomicAdd(&s_cnt[e], 1);
+        }
         __syncthreads();
         const int c = tid < E ? s_cnt[tid] : 0;
         int off;
@@ -788,6 +860,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         }
         __syncthreads();
     }
+    DF_MARK(6);
 
     // ---- C: gate/up + SwiGLU.  A grid barrier separates C from D, so each phase
     // is balanced on its own: every CTA takes an equal share of the 16-row
@@ -882,6 +955,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         for (; s < nC; ++s) {
             const int b = s % DF_NBUF;
             if (!mbar_wait(&full[warp * DF_NBUF + b], (uint32_t)(s / DF_NBUF) & 1u, 4, s)) { wok = false; break; }
+            if (s == 0) DF_MARK(7);
             const int u = ub + s, lt = u / NCH, ch = u % NCH, gt = r0 + lt, ui = gt / tiles_e;
             const bool valid = rt.u_sl[ui] >= 0;
             DfCRegs<BGU> cr;
@@ -909,6 +983,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         }
     }
     const bool cok = __syncthreads_and(wok && alive) != 0;
+    DF_MARK(8);
     // finish the tiles: sum the partials of the warps that covered each tile (in
     // warp order), SwiGLU, round h to bf16 and store it for every pair of the expert
     if (cok) {
@@ -930,10 +1005,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             a.hB[(size_t)pos * I + frag_pos(r16 * 16 + row)] = f32_to_bf16_bits(h);
         }
     }
+    DF_MARK(9);
     {
         const bool gb = grid_barrier(a.bar, 2u, 2, a.spin_limit);
         alive = __syncthreads_and(cok && gb) != 0;
     }
+    DF_MARK(10);
 
     // ---- D: down projection of this CTA's feature tiles for every selected
     // expert (warp w takes experts w, w + 16, ...), then the combine.
@@ -959,6 +1036,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             hsum[it] = sum;
         }
         __syncthreads();
+        DF_MARK(11);
     }
     if (alive) {
         const int g = lane >> 2, q = lane & 3;
@@ -987,6 +1065,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             }
         }
         alive = __syncthreads_and(wok) != 0;
+        DF_MARK(12);
         if (alive)
             for (int u = tid; u < nftc * T * DF_FT; u += DF_THREADS) {
                 const int rr = u / (T * DF_FT), t = (u / DF_FT) % T, fl = u % DF_FT;
@@ -994,10 +1073,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                 float sum = 0.f;
                 for (int j = 0; j < k; ++j) sum += ypair[((size_t)rr * P + rt.inv[t * k + j]) * DF_FT + fl];
                 if (a.residual) sum = bf16_bits_to_f32(a.x[(size_t)t * H + f]) + sum;
-                a.out[(size_t)t * H + f] = f32_to_bf16_bits(sum);
+                if (a.hout) a.hout[(size_t)t * H + f] = sum;
+                else a.out[(size_t)t * H + f] = f32_to_bf16_bits(sum);
             }
     }
     // On an error path, wait (bounded) for this warp's copies still in flight
     // before the CTA's shared memory goes away.
     for (int r = s; r < issued; ++r) mbar_wait(&full[warp * DF_NBUF + r % DF_NBUF], (uint32_t)(r / DF_NBUF) & 1u, 8, r);
+    DF_MARK(13);
 }

@@ -24,7 +24,7 @@ inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
     size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, wsplit,
-        xn, slow, total;
+        xn, slow, hout, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -57,6 +57,7 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.wsplit = put(small ? 0 : (size_t)3 * E * H * 2);        // chunk router: W_r as three bf16 planes
     w.xn = put(small ? 0 : (size_t)T * 4);                     // chunk router: ||x_t|| per token
     w.slow = put(small ? 0 : (size_t)(T + 4) * 4);             // chunk top-k: [count, tokens...] left to the slow pass
+    w.hout = put(small ? (size_t)T * H * 4 : 0);               // fused decode + steering: fp32 output rows
     w.total = o;
     return w;
 }
@@ -75,8 +76,12 @@ constexpr int kDfMaxH = 2560;           // largest H the fused decode kernel sta
 
 inline void stage(int i, cudaStream_t st) {
     std::lock_guard<std::mutex> g(g_mu);
-    // external: inside a stream capture this becomes an event-record node of the graph
-    if ((int)g_stage_ev.size() > i) cudaEventRecordWithFlags(g_stage_ev[i], st, cudaEventRecordExternal);
+    if ((int)g_stage_ev.size() <= i) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(g_stage_ev[i], st, cudaEventRecordExternal);  // an event-record node of the graph
+    else
+        cudaEventRecord(g_stage_ev[i], st);
 }
 
 inline void count(int n) { g_launches += (uint64_t)n; }
@@ -296,6 +301,7 @@ struct LayerCall {
     const float* W;
     const float* b;
     int E, k, residual;
+    const float* steer;
     uint16_t* out;
     uint32_t* hist;
     const moe_route_out* ro;
@@ -311,7 +317,7 @@ int check_layer(const LayerCall& c, bool prefill) {
     if (rc) return rc;
     if (c.L < 1 || c.layer < 0 || c.layer >= c.L) return MOE_ERR_RANGE;
     if (!c.arena || !c.slot_table || !c.out) return MOE_ERR_ARG;
-    if (!aligned(c.arena, 256) || !aligned(c.out, 16)) return MOE_ERR_ARG;
+    if (!aligned(c.arena, 256) || !aligned(c.out, 16) || !aligned(c.steer, 16)) return MOE_ERR_ARG;
     const size_t xb = (size_t)c.T * c.d->H * 2;
     const uintptr_t x0 = reinterpret_cast<uintptr_t>(c.x), o0 = reinterpret_cast<uintptr_t>(c.out);
     if (c.T > 0 && x0 < o0 + xb && o0 < x0 + xb) return MOE_ERR_ARG;
@@ -392,8 +398,10 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = d->n_slots; a.slot_bytes = d->slot_bytes;
     for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
     a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.residual;
+    a.bits_gate = d->bits_gate; a.bits_up = d->bits_up; a.bits_down = d->bits_down;
     a.epc = epc;
     a.x = c.x; a.W = c.W; a.b = c.b; a.out = c.out; a.hist = c.hist;
+    a.hout = c.steer ? reinterpret_cast<float*>(c.ws + L.hout) : nullptr;
     a.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
     a.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
     a.offsets = (ro && ro->expert_offsets) ? ro->expert_offsets : reinterpret_cast<int32_t*>(c.ws + L.offsets);
@@ -433,6 +441,11 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
         case 2408: e = launch_fused<2, 4, 8>(tm, a, grid, dyn, c.st); break;
         default: e = launch_fused<2, 2, 16>(tm, a, grid, dyn, c.st); break;
     }
+    if (e == cudaSuccess && c.steer) {  // steering: the rows leave the kernel in fp32, one block per token finishes them
+        k_combine_steer<float><<<c.T, STEER_THREADS, H * 4, c.st>>>(nullptr, nullptr, nullptr, a.hout, c.T, H, c.k, 0,
+                                                                    c.steer, c.out);
+        count(1);
+    }
     for (int i = 1; i < 5; ++i) stage(i, c.st);  // one kernel: the stages collapse onto its end
     count(1);
     return e == cudaSuccess ? cuda_rc(cudaGetLastError()) : MOE_ERR_CUDA;
@@ -469,8 +482,12 @@ int run_decode(const LayerCall& c) {
     if (d->bits_down == 4) launch_down<4>(a, umax, c.T, c.st);
     else launch_down<2>(a, umax, c.T, c.st);
     stage(3, c.st);
-    k_combine<float><<<dim3((d->H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
-        c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, d->H, c.k, c.residual, c.out);
+    if (c.steer)
+        k_combine_steer<float><<<c.T, STEER_THREADS, d->H * 4, c.st>>>(
+            c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), nullptr, c.T, d->H, c.k, c.residual, c.steer, c.out);
+    else
+        k_combine<float><<<dim3((d->H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+            c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, d->H, c.k, c.residual, c.out);
     stage(4, c.st);
     count(3);
     return cuda_rc(cudaGetLastError());
@@ -533,8 +550,12 @@ int run_prefill(const LayerCall& c) {
     if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, a, H / PF_BM, mg2, nt, c.st);
     else launch_gemm<1, 2, 2>(th, a, H / PF_BM, mg2, nt, c.st);
     stage(3, c.st);
-    k_combine_bf16x8<<<dim3((H / 8 + 127) / 128, c.T), 128, 0, c.st>>>(
-        c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);
+    if (c.steer)
+        k_combine_steer<uint16_t><<<c.T, STEER_THREADS, H * 4, c.st>>>(
+            c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), nullptr, c.T, H, c.k, c.residual, c.steer, c.out);
+    else
+        k_combine_bf16x8<<<dim3((H / 8 + 127) / 128, c.T), 128, 0, c.st>>>(
+            c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.residual, c.out);
     stage(4, c.st);
     count(4);
     return cuda_rc(cudaGetLastError());
@@ -637,10 +658,10 @@ int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, con
 
 static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L,
                    int layer, const uint16_t* x, int T, const float* router_w, const float* router_bias, int E,
-                   int top_k, int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
-                   size_t ws_bytes, void* stream) {
+                   int top_k, int residual, const float* steer, uint16_t* out, uint32_t* hist,
+                   const moe_route_out* route_out, void* ws, size_t ws_bytes, void* stream) {
     LayerCall c{desc, static_cast<const uint8_t*>(arena), slot_table, L, layer, x, T, router_w, router_bias, E,
-                top_k, residual, out, hist, route_out, static_cast<uint8_t*>(ws), ws_bytes,
+                top_k, residual, steer, out, hist, route_out, static_cast<uint8_t*>(ws), ws_bytes,
                 static_cast<cudaStream_t>(stream)};
     int rc = check_layer(c, prefill);
     if (rc) return rc;
@@ -652,17 +673,17 @@ static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, 
 
 int moe_forward_decode(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L, int layer,
                        const uint16_t* x, int T, const float* router_w, const float* router_bias, int E, int top_k,
-                       int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
-                       size_t ws_bytes, void* stream) {
-    return forward(false, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, out,
+                       int residual, const float* steer, uint16_t* out, uint32_t* hist, const moe_route_out* route_out,
+                       void* ws, size_t ws_bytes, void* stream) {
+    return forward(false, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, steer, out,
                    hist, route_out, ws, ws_bytes, stream);
 }
 
 int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L, int layer,
                         const uint16_t* x, int T, const float* router_w, const float* router_bias, int E, int top_k,
-                        int residual, uint16_t* out, uint32_t* hist, const moe_route_out* route_out, void* ws,
-                        size_t ws_bytes, void* stream) {
-    return forward(true, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, out,
+                        int residual, const float* steer, uint16_t* out, uint32_t* hist, const moe_route_out* route_out,
+                        void* ws, size_t ws_bytes, void* stream) {
+    return forward(true, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, steer, out,
                    hist, route_out, ws, ws_bytes, stream);
 }
 
@@ -687,6 +708,88 @@ int moe_rank_experts(const uint32_t* hist_host, int L, int E, uint16_t* pairs_ou
         pairs_out[2 * r + 1] = (uint16_t)(order[r] % E);
     }
     return MOE_OK;
+}
+
+// ---------------------------------------------------------------- expert profile (STRP v1)
+
+int64_t moe_profile_bytes(int n_pairs, int L, int E) {
+    if (L < 1 || E < 1 || L > 65535 || E > 65535 || n_pairs < 0 || (int64_t)n_pairs > (int64_t)L * E) return -1;
+    return 4 + 5 * 4 + (int64_t)n_pairs * 4 + (int64_t)L * E * 4;
+}
+
+namespace {
+inline void put_u32(uint8_t* p, uint32_t v) { for (int i = 0; i < 4; ++i) p[i] = (uint8_t)(v >> (8 * i)); }
+inline void put_u16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
+inline uint32_t get_u32(const uint8_t* p) { return p[0] | (p[1] << 8) | (p[2] << 16) | ((uint32_t)p[3] << 24); }
+inline uint16_t get_u16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+}  // namespace
+
+int64_t moe_profile_write(const uint16_t* pairs, int n_pairs, int L, int E, uint8_t* buf, size_t buf_bytes) {
+    const int64_t need = moe_profile_bytes(n_pairs, L, E);
+    if (need < 0) return MOE_ERR_RANGE;
+    if (!buf) return need;
+    if (!pairs && n_pairs > 0) return MOE_ERR_ARG;
+    if (buf_bytes < (size_t)need) return MOE_ERR_WS;
+    std::vector<int32_t> inv((size_t)L * E, -1);
+    for (int r = 0; r < n_pairs; ++r) {
+        const int l = pairs[2 * r], e = pairs[2 * r + 1];
+        if (l >= L || e >= E || inv[(size_t)l * E + e] >= 0) return MOE_ERR_ARG;  // out of range or ranked twice
+        inv[(size_t)l * E + e] = r;
+    }
+    uint8_t* p = buf;
+    p[0] = 'S'; p[1] = 'T'; p[2] = 'R'; p[3] = 'P';
+    put_u32(p + 4, 1);                          // version
+    put_u32(p + 8, (uint32_t)L);                // layers
+    put_u32(p + 12, (uint32_t)E);               // experts per layer
+    put_u32(p + 16, (uint32_t)n_pairs);         // ranked pairs
+    put_u32(p + 20, (uint32_t)((int64_t)L * E));  // entries of the inverse tables
+    p += 24;
+    for (int r = 0; r < n_pairs; ++r, p += 4) {
+        put_u16(p, pairs[2 * r]);
+        put_u16(p + 2, pairs[2 * r + 1]);
+    }
+    for (size_t i = 0; i < inv.size(); ++i, p += 4) put_u32(p, (uint32_t)inv[i]);
+    return need;
+}
+
+int moe_profile_read(const uint8_t* buf, size_t bytes, int* L, int* E, int* n_pairs, uint16_t* pairs,
+                     int32_t* inverse) {
+    if (!buf || !L || !E || !n_pairs) return MOE_ERR_ARG;
+    if (bytes < 24 || buf[0] != 'S' || buf[1] != 'T' || buf[2] != 'R' || buf[3] != 'P') return MOE_ERR_SHAPE;
+    if (get_u32(buf + 4) != 1) return MOE_ERR_SHAPE;
+    const uint32_t l = get_u32(buf + 8), e = get_u32(buf + 12), n = get_u32(buf + 16), ent = get_u32(buf + 20);
+    if (l < 1 || e < 1 || l > 65535 || e > 65535 || (uint64_t)n > (uint64_t)l * e || (uint64_t)ent != (uint64_t)l * e)
+        return MOE_ERR_SHAPE;
+    if ((int64_t)bytes != moe_profile_bytes((int)n, (int)l, (int)e)) return MOE_ERR_SHAPE;
+    *L = (int)l; *E = (int)e; *n_pairs = (int)n;
+    const uint8_t* p = buf + 24;
+    for (uint32_t r = 0; r < n; ++r, p += 4) {
+        const uint16_t pl = get_u16(p), pe = get_u16(p + 2);
+        if (pl >= l || pe >= e) return MOE_ERR_SHAPE;
+        if (pairs) { pairs[2 * r] = pl; pairs[2 * r + 1] = pe; }
+    }
+    for (uint64_t i = 0; i < ent; ++i, p += 4) {
+        const int32_t v = (int32_t)get_u32(p);
+        if (v < -1 || v >= (int32_t)n) return MOE_ERR_SHAPE;
+        if (inverse) inverse[i] = v;
+    }
+    return MOE_OK;
+}
+
+double moe_profile_hit_rate(const uint16_t* pairs, int n_pairs, int L, int E, int slots, const uint32_t* hist) {
+    if (!hist || (!pairs && n_pairs > 0) || L < 1 || E < 1 || n_pairs < 0 || slots < 0) return -1.0;
+    const int use = std::min(slots, n_pairs);
+    uint64_t total = 0, hit = 0;
+    for (int64_t i = 0; i < (int64_t)L * E; ++i) total += hist[i];
+    std::vector<char> cached((size_t)L * E, 0);
+    for (int r = 0; r < use; ++r) {
+        const int l = pairs[2 * r], e = pairs[2 * r + 1];
+        if (l >= L || e >= E) return -1.0;
+        const size_t i = (size_t)l * E + e;
+        if (!cached[i]) hit += hist[i];
+        cached[i] = 1;
+    }
+    return total ? (double)hit / (double)total : 0.0;
 }
 
 int moe_last_device_error(void* stream) {
@@ -722,6 +825,7 @@ size_t moe_workspace_offset(int T, int E, int top_k, int H, int I, int field) {
     switch (field) {
         case MOE_WS_FAST_LOGITS: return L.logit;
         case MOE_WS_PAIR_OUT: return L.y;
+        case MOE_WS_SLOW_COUNT: return L.slow;
         default: return (size_t)-1;
     }
 }
@@ -739,6 +843,13 @@ int moe_timeout_site(void* stream) {
     if (cudaMemcpyToSymbol(g_moe_where, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
     return v;
 }
+
+#ifdef MOE_PROBE
+// Measurement builds only: the fused decode kernel's phase timestamps of the last launch.
+int moe_probe_read(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_df_probe, sizeof(g_df_probe)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 const char* moe_strerror(int code) {
     switch (code) {

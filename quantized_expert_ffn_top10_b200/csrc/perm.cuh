@@ -27,12 +27,22 @@ struct PermArgs {
     int layer;
 };
 
+// Expert of pair p.  The top-k only writes valid experts; an index outside
+// [0, E) would mean a library fault, and is counted as expert 0 (the same in
+// both passes, so the grouping stays a bijection) with MOE_ERR_RANGE latched.
+__device__ __forceinline__ int pair_expert(const PermArgs& a, int p) {
+    const int e = a.idx[p];
+    if ((unsigned)e < (unsigned)a.E) return e;
+    moe_set_status(MOE_ERR_RANGE);
+    return 0;
+}
+
 __global__ void __launch_bounds__(PERM_CHUNK) k_perm_count(PermArgs a) {
     __shared__ int cnt[MOE_MAX_E];
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     int p = blockIdx.x * PERM_CHUNK + threadIdx.x;
-    if (p < a.P) atomicAdd(&cnt[a.idx[p]], 1);
+    if (p < a.P) atomicAdd(&cnt[pair_expert(a, p)], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.chunk_cnt[(size_t)blockIdx.x * a.E + e] = cnt[e];
 }
@@ -117,7 +127,7 @@ __global__ void __launch_bounds__(PERM_CHUNK) k_perm_scatter(PermArgs a) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int p = blockIdx.x * PERM_CHUNK + threadIdx.x;
     const bool valid = p < a.P;
-    const int e = valid ? a.idx[p] : -1;
+    const int e = valid ? pair_expert(a, p) : -1;
     const unsigned grp = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(grp & ((1u << lane) - 1));
     const int leader = __ffs(grp) - 1;

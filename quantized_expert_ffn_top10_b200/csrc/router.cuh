@@ -208,6 +208,20 @@ __device__ __forceinline__ double warp_min_d(double v) {
     return v;
 }
 
+// The selection order of logits is total: a NaN logit ranks as -inf (below
+// every number; ties, as every tie, go to the lower expert index), and an
+// error bound that is not a number becomes +inf, against which nothing
+// certifies.  Non-finite inputs therefore still give k valid, distinct experts.
+__device__ __forceinline__ double order_val(double v) { return isnan(v) ? -INFINITY : v; }
+__device__ __forceinline__ double order_bnd(double d) { return isnan(d) ? INFINITY : d; }
+
+// Ends of the interval [v - d, v + d] that holds an exact logit.  An infinite
+// bound leaves the value unknown, so its interval is the whole line (plain
+// arithmetic would give inf - inf = NaN there, and a NaN end would silently
+// drop out of the comparisons, maxima and minima that use it).
+__device__ __forceinline__ double lo_end(double v, double d) { return isinf(d) ? -INFINITY : v - d; }
+__device__ __forceinline__ double hi_end(double v, double d) { return isinf(d) ? INFINITY : v + d; }
+
 // The definition: fp64, sequential over h, then + b (one thread).
 __device__ __forceinline__ double logit_fp64_exact(const TopkArgs& a, int t, int e) {
     const uint16_t* xr = a.x + (size_t)t * a.H;
@@ -240,8 +254,8 @@ __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int
     const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
     const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
     bool ok = true;
-    if (lane < k && lane + 1 < M) ok = (cval - cbnd) > (nv + nb);
-    if (lane == k - 1) ok = ok && (rest == -INFINITY || (cval - cbnd) > rest);
+    if (lane < k && lane + 1 < M) ok = lo_end(cval, cbnd) > hi_end(nv, nb);
+    if (lane == k - 1) ok = ok && (rest == -INFINITY || lo_end(cval, cbnd) > rest);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -309,15 +323,16 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             double B;
             float f;
             if (F64) {
-                v[i] = static_cast<const double*>(a.logit)[(size_t)t * E + e];
+                v[i] = order_val(static_cast<const double*>(a.logit)[(size_t)t * E + e]);
                 f = (float)v[i];
             } else {
                 f = static_cast<const float*>(a.logit)[(size_t)t * E + e];
+                if (isnan(f)) f = -INFINITY;
                 v[i] = (double)f;
             }
             if (MODE == 1) B = a.absum[(size_t)t * E + e] * (1.0 + 1e-9);
             else B = ((double)xnorm * (double)a.wnorm[e] + (a.b ? fabs((double)a.b[e]) : 0.0)) * 1.001;
-            dl[i] = B * (a.gfast + g_or) + 1e-300;
+            dl[i] = order_bnd(B * (a.gfast + g_or) + 1e-300);
             const uint32_t u = __float_as_uint(f);
             key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         } else {
@@ -416,7 +431,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     double rest = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-        if (!((taken >> i) & 1u)) rest = fmax(rest, v[i] + dl[i]);
+        if (!((taken >> i) & 1u)) rest = fmax(rest, hi_end(v[i], dl[i]));
     rest = warp_max_d(rest);
 
     // 2) certified on the fast values?
@@ -437,7 +452,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     if (MODE == 0) {
         const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
         const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
-        const bool pairbad = lane < k && lane + 1 < MC && !((cval - cbnd) > (nv + nb));
+        const bool pairbad = lane < k && lane + 1 < MC && !(lo_end(cval, cbnd) > hi_end(nv, nb));
         const bool prevbad = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0 && lane > 0;
         const unsigned need = __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad));
         const int NR = __popc(need);
@@ -471,8 +486,8 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
                     const double s = warp_sum_d(acc[j]), sa = warp_sum_d(ab[j]);
                     const double bb = a.b ? (double)a.b[ej[j]] : 0.0;
                     if (lane == lj[j]) {
-                        cval = s + bb;
-                        cbnd = (sa + fabs(bb)) * (1.0 + 1e-9) * (g_par + g_or) + 1e-300;
+                        cval = order_val(s + bb);
+                        cbnd = order_bnd((sa + fabs(bb)) * (1.0 + 1e-9) * (g_par + g_or) + 1e-300);
                     }
                 }
             }
@@ -484,18 +499,18 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     }
     // 4) exact: every expert whose upper end reaches theta (the lowest lower
     //    end among the k best) is evaluated by the definition itself
-    const double th = warp_min_d(lane < k ? cval - cbnd : INFINITY);
+    const double th = warp_min_d(lane < k ? lo_end(cval, cbnd) : INFINITY);
     int nc = 0;
     for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
         // the step-1 candidates (marked taken) are always kept
-        const bool in = (e < E) && ((((taken >> i) & 1u) != 0) || v[i] + dl[i] >= th);
+        const bool in = (e < E) && ((((taken >> i) & 1u) != 0) || hi_end(v[i], dl[i]) >= th);
         const unsigned m = __ballot_sync(0xffffffffu, in);
         if (in) cs[nc + __popc(m & ((1u << lane) - 1))] = e;
         nc += __popc(m);
     }
     __syncwarp();
-    for (int c = lane; c < nc; c += 32) cvs[c] = logit_fp64_exact(a, t, cs[c]);
+    for (int c = lane; c < nc; c += 32) cvs[c] = order_val(logit_fp64_exact(a, t, cs[c]));
     __syncwarp();
     double l0 = 0.0, z = 0.0, mine = 0.0;
     for (int j = 0; j < k; ++j) {
@@ -512,8 +527,15 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         }
         __syncwarp();
         if (lane == 0) {
-            cs[bc] = -1;  // taken
-            idx_out[j] = be;
+            // at least k candidates and a total order: bc is always found; the
+            // guard only keeps a library fault from writing outside the arrays
+            if (bc >= 0 && be < E) {
+                cs[bc] = -1;  // taken
+                idx_out[j] = be;
+            } else {
+                idx_out[j] = 0;
+                moe_set_status(MOE_ERR_RANGE);
+            }
         }
         __syncwarp();
         if (j == 0) l0 = bv;

@@ -38,12 +38,12 @@ def test_workspace_bytes_grows_with_T(lib):
 
 
 def _fwd(fn, desc, T=5, E=512, k=10, L=1, layer=0, x=FAKE, out=FAKE + (1 << 16), ws=FAKE * 64,
-         ws_bytes=None, arena=FAKE * 128, W=FAKE * 4):
+         ws_bytes=None, arena=FAKE * 128, W=FAKE * 4, steer=None):
     d = M.as_desc(desc) if desc is not None else None
     if ws_bytes is None:
         ws_bytes = 1 << 40
-    return fn(ctypes.byref(d) if d is not None else None, arena, FAKE * 8, L, layer, x, T, W, None, E, k, 1, out,
-              None, None, ws, ws_bytes, None)
+    return fn(ctypes.byref(d) if d is not None else None, arena, FAKE * 8, L, layer, x, T, W, None, E, k, 1, steer,
+              out, None, None, ws, ws_bytes, None)
 
 
 @pytest.mark.parametrize("which", ["decode", "prefill"])
@@ -71,6 +71,7 @@ def test_host_checks(lib, which):
     assert _fwd(fn, d, arena=FAKE * 128 + 16) == M.MOE_ERR_ARG
     assert _fwd(fn, d, out=FAKE + 64) == M.MOE_ERR_ARG       # overlaps x
     assert _fwd(fn, d, ws_bytes=1024) == M.MOE_ERR_WS
+    assert _fwd(fn, d, steer=FAKE * 2 + 4) == M.MOE_ERR_ARG  # steering vector not 16-byte aligned
 
 
 def test_prefill_needs_tile_multiples(lib):

@@ -108,7 +108,9 @@ def test_decode_missing_slot_contributes_zero(cuda_ok):
 
 def test_decode_stack_teacher_forced(cuda_ok):
     """48 layers x 256 experts, 2/2/4-bit, Zipf bias: the oracle chains its own
-    bf16 outputs; every layer of the library gets the oracle's input."""
+    bf16 outputs; every layer of the library gets the oracle's input.  Each
+    layer runs twice: with the residual (the chain) and without it, so that the
+    MoE part, a small fraction of x in this stable chain, is checked on its own."""
     import torch
     cfg = S.config("decode_stack")
     wl = Workload(cfg)
@@ -118,12 +120,15 @@ def test_decode_stack_teacher_forced(cuda_ok):
     distinct = []
     for layer in range(cfg.L):
         out, res = run_layer(wl, layer, x, prefill=False, hist=hist)
-        ref = wl.oracle_layer(layer, x)
+        moe, _ = run_layer(wl, layer, x, prefill=False, residual=False)
+        ref = wl.oracle_layer(layer, x, residual=False)
         counts = check_routing(res, ref["idx"], ref["w"], cfg.E)
         O.hist_add(counts, layer, ref_hist)
-        assert_out_close(out, ref["out_f64"])
+        assert_out_close(moe, ref["out_f64"])
+        xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        assert_out_close(out, xf + ref["out_f64"])  # the oracle's residual form: x + sum_j w_j y_j
         distinct.append(int((counts > 0).sum()))
-        x = ref["out"]
+        x = np.array([[O.double_to_bf16(v) for v in row] for row in xf + ref["out_f64"]], np.uint16)
     assert np.array_equal(hist.cpu().numpy().view(np.uint32), ref_hist)
     assert max(distinct) <= cfg.T * cfg.top_k
 

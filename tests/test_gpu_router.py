@@ -168,3 +168,31 @@ def test_route_histogram_entry_point(cuda_ok):
     got = hist.cpu().numpy().view(np.uint32)
     assert np.array_equal(got, ref)
     assert got.sum() == k * sum(T for _, T, _ in calls)
+
+
+def test_profile_from_device_histogram(cuda_ok):
+    """The expert-profile pipeline on the device: routing counts of 3 windows
+    per layer of the 48 x 256 stack accumulated by moe_route_histogram, ranked
+    by moe_rank_experts and written as STRP v1 - byte-identical to the
+    oracle's file from its own counts."""
+    import torch
+    import quantized_expert_ffn_top10_b200 as M
+    from oracle import profile as OP
+    cfg = S.config("decode_stack")
+    L, E, k = cfg.L, cfg.E, cfg.top_k
+    hist = torch.zeros((L, E), dtype=torch.int32, device="cuda")
+    ref = np.zeros((L, E), np.uint32)
+    for layer in range(L):
+        W, b = S.gen_router(cfg, layer), S.gen_bias(cfg, layer)
+        for off in range(3):
+            x = S.gen_x(cfg, 5, stream_offset=200 + 3 * layer + off)
+            res = _route(x, W, b, k)
+            M.moe_route_histogram(torch.from_numpy(res["expert_offsets"]).cuda(), E, L, layer, hist)
+            idx, _ = O.topk(O.router_logits(x, W, b), k)
+            counts, *_ = O.permutation(idx, E)
+            O.hist_add(counts, layer, ref)
+    torch.cuda.synchronize()
+    got = hist.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, ref)
+    pairs = M.moe_rank_experts(got)
+    assert M.moe_profile_write(pairs, L, E) == OP.profile_bytes(O.rank(ref).tolist(), L, E)

@@ -117,3 +117,53 @@ def test_token_subset_matches_full_run():
         assert np.array_equal(sub["out"][t], full["out"][t])
         assert np.array_equal(sub["idx"][t], full["idx"][t])
     assert np.all(sub["out"][1] == 0)
+
+
+def _steer_setup():
+    cfg, d, arena, st, x, W = _tiny()
+    rng = np.random.default_rng(71)
+    v = rng.standard_normal(cfg.H)
+    v = (v / np.linalg.norm(v)).astype(np.float32)
+    return cfg, d, arena, st, x, W, v
+
+
+def test_steer_parallel_and_orthogonal_rows_closed_form():
+    """With every expert at zero scale the layer output is x itself; for the
+    unit direction e_5, a row equal to a multiple of e_5 projects to exactly 0
+    and a row with a zero 5th entry is unchanged."""
+    cfg, d, arena, st, x, W = _tiny()
+    z = arena.copy()
+    for s in range(d.n_slots):
+        base = s * d.slot_bytes
+        for m in range(3):
+            rows, K = S.matrix_shape(d.H, d.I, m)
+            z[base + d.off_scales[m]:base + d.off_scales[m] + rows * (K // 32) * 2] = 0
+    v = np.zeros(cfg.H, np.float32)
+    v[5] = 1.0
+    xs = np.zeros_like(x)
+    xs[0, 5] = S.f32_to_bf16_bits(np.array([-3.25], np.float32))[0]           # parallel to v
+    xs[1] = x[1]
+    xs[1, 5] = 0                                                              # orthogonal to v
+    xs[2:] = x[2:]
+    res = O.moe_layer(d, z, st, 1, 0, xs, W, None, cfg.top_k, steer=v)
+    assert np.all(res["out_f64"][0] == 0.0)
+    assert np.array_equal(res["out"][1], xs[1])
+
+
+def test_steer_invariants_on_the_tiny_layer():
+    """Against the unsteered layer output h, with s = h . v and n = v . v (v is
+    an fp32 rounding of a unit vector, so n = 1 only to ~1e-7):
+    out . v = s (1 - n), ||out||^2 = ||h||^2 - 2 s^2 + s^2 n, and a second
+    projection moves the row only by s (1 - n) v."""
+    cfg, d, arena, st, x, W, v = _steer_setup()
+    h = O.moe_layer(d, arena, st, 1, 0, x, W, None, cfg.top_k)["out_f64"]
+    out = O.moe_layer(d, arena, st, 1, 0, x, W, None, cfg.top_k, steer=v)["out_f64"]
+    vd = v.astype(np.float64)
+    n = vd @ vd
+    assert abs(n - 1) < 1e-6
+    for t in range(cfg.T):
+        s = h[t] @ vd
+        tol = 1e-13 * np.linalg.norm(h[t]) ** 2
+        assert abs(out[t] @ vd - s * (1 - n)) <= 1e-13 * np.linalg.norm(h[t])
+        assert abs(out[t] @ out[t] - (h[t] @ h[t] - 2 * s * s + s * s * n)) <= tol
+        assert np.allclose(O.steer(out[t], v), out[t] - s * (1 - n) * vd, rtol=0, atol=1e-13 * np.linalg.norm(h[t]))

@@ -402,3 +402,19 @@ def test_expert_ffn_rows_matches_per_element_oracle():
             Wm = O.dequant_matrix(slot, d, m)
             for r, c in [(0, 0), (rows - 1, K - 1), (rows // 2, 33), (1, K // 2 + 7)]:
                 assert Wm[r, c] == O.dequant(slot, d, m, r, c)
+
+
+def test_topk_non_finite_logits_total_order():
+    """NaN logits rank as -inf (below every number, ties by lower index) and
+    weigh 0 when selected next to a finite maximum; +inf ranks first."""
+    nan, inf = float("nan"), float("inf")
+    lg = np.array([[nan, 1.0, -inf, 0.5, nan, 2.0],
+                   [nan, nan, nan, nan, nan, nan],
+                   [0.0, inf, 1.0, inf, -1.0, nan]])
+    idx, w = O.topk(lg, 4)
+    assert idx[0].tolist() == [5, 1, 3, 0]            # the NaN at 0 ties -inf at 2 and wins by index
+    assert w[0, 3] == 0.0 and np.isclose(w[0, :3].sum(), 1.0)
+    assert idx[1].tolist() == [0, 1, 2, 3]            # all NaN: the lowest indices
+    assert np.all(np.isnan(w[1]))
+    assert idx[2].tolist() == [1, 3, 2, 0]
+    assert np.all(np.isnan(w[2]))                     # exp(inf - inf)

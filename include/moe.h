@@ -259,8 +259,10 @@ const char* moe_strerror(int code);
  * forward call records the caller's CUDA events (cudaEvent_t, created with
  * timing enabled) on its stream at the stage boundaries: events[0] before the
  * router, [1] after grouping, [2] after the first expert stage (gate/up),
- * [3] after the second (down), [4] after the combine.  n = 0 (or events =
- * NULL) turns it off.  The setting is process-wide and read at call time, so
+ * [3] after the second (down), [4] after the combine; a call that runs as
+ * one fused kernel records only [0] before it and [1] after it (each record
+ * in a graph costs microseconds of device time).  n = 0 (or events = NULL)
+ * turns it off.  The setting is process-wide and read at call time, so
  * a call captured into a CUDA graph records into the events set at capture.
  * moe_launch_count(): kernels this process has launched through the library
  * (host-side counter; launches replayed from a captured graph are not added).

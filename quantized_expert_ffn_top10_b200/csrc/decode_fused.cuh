@@ -42,7 +42,8 @@
 // CTA records the global timer at the phase boundaries.  Compiled out
 // otherwise.
 #ifdef MOE_PROBE
-__device__ unsigned long long g_df_probe[160][16];
+#define DF_WARPS_PROBE 16
+__device__ unsigned long long g_df_probe[160][24];
 #define DF_MARK(i)                                                                  \
     do {                                                                            \
         if (threadIdx.x == 0 && blockIdx.x < 160) {                                 \
@@ -51,9 +52,21 @@ __device__ unsigned long long g_df_probe[160][16];
             g_df_probe[blockIdx.x][i] = t_;                                         \
         }                                                                           \
     } while (0)
+// per warp: cycles waiting for C units, computing them, the same for D, units of each
+#define DF_NWP 10
+__device__ unsigned long long g_df_wprobe[160][DF_WARPS_PROBE][DF_NWP];
+#define DF_CLK(v) unsigned long long v = clock64()
+#define DF_WACC(slot, val) \
+    do { if ((threadIdx.x & 31) == 0 && blockIdx.x < 160) g_df_wprobe[blockIdx.x][threadIdx.x >> 5][slot] += (val); } while (0)
 #else
 #define DF_MARK(i) \
     do {           \
+    } while (0)
+#define DF_CLK(v) \
+    do {          \
+    } while (0)
+#define DF_WACC(slot, val) \
+    do {               \
     } while (0)
 #endif
 
@@ -69,6 +82,7 @@ __device__ unsigned long long g_df_probe[160][16];
 #define DF_SMEM_LIMIT (227 * 1024)
 #define DF_BAR_WORDS (32 * 18)  // grid barrier: 16 group counters, the top counter, the flag
 #define DF_NREP 8          // copies of the (logit, bound) records that phase B reads
+#define DF_CAND_BYTES 640  // phase-B candidate scratch of one token: 32 experts, 32 values + 32 bounds
 
 // Shared-memory layout, computed on the host (df_plan) and passed in; offsets
 // are from the 1024-byte aligned base of dynamic shared memory.
@@ -80,8 +94,10 @@ struct DfPlan {
     int route_off, stab_off, bar_off, total;
     // phase A (code ring, free then): x rows, W_r rows, per-warp sums, x block sums
     int a_ws_off, a_sp_off, a_w2_off, a_xp_off;
-    // phase B (code ring): per-token scratch, expert counts and offsets
-    int b_cnt_off, b_off_off;
+    // phase B (code ring): the (logit, bound) records, their keys, per-token candidate
+    // scratch (32 experts, 64 doubles), and the exact fallback's scratch: the token's
+    // own record row when it is large enough (b_fb_off < 0), else a region of its own
+    int b_rec_off, b_key_off, b_cand_off, b_fb_off, b_fb_stride;
 };
 
 struct DecodeFusedArgs {
@@ -108,6 +124,7 @@ struct DecodeFusedArgs {
     double* logit;           // [T][E] workspace
     float* wnorm;            // [E] upper bounds of ||W[e]||_2 (workspace)
     double2* rec;            // [DF_NREP][T][E] (logit, error bound): CTA c reads copy c % DF_NREP
+    uint2* reck;             // [DF_NREP][T][E] (key32 of the fp32 logit, upper end rounded up to fp32)
     uint16_t* hB;            // [P][I] bf16, MMA-fragment order within each 32-block
     unsigned int* bar;       // grid barrier counters and flag, DF_BAR_WORDS words (zeroed before launch)
     unsigned spin_limit;     // polling bound of the grid barriers (MOE_SPIN_LIMIT; lowered only by a test)
@@ -165,12 +182,18 @@ __host__ inline bool df_plan(DfPlan& p, int T, int P, int E, int H, int I, int b
     p.a_sp_off = df_al(p.a_ws_off + epc * (4 * H + 16), 128);
     p.a_w2_off = p.a_sp_off + DF_WARPS * 64 * 8;
     p.a_xp_off = p.a_w2_off + DF_WARPS * DF_TN * 4;
-    // phase B inside the code ring: per-token scratch (6 KB each), counts, offsets
-    p.b_cnt_off = DF_TN * MOE_MAX_E * 12;
-    p.b_off_off = p.b_cnt_off + MOE_MAX_E * 4;
+    // phase B inside the code ring: the records, their keys, the candidate scratch
+    // [T][32 ints | 64 doubles] and, for small E, the fallback scratch
+    // [T][max(E,32) ints | max(E,64) doubles]
+    p.b_rec_off = 0;
+    p.b_key_off = T * E * 16;
+    p.b_cand_off = p.b_key_off + T * E * 8;
+    p.b_fb_stride = df_al(4 * std::max(E, 32), 8) + 8 * std::max(E, 64);
+    p.b_fb_off = p.b_fb_stride <= 16 * E ? -1 : p.b_cand_off + T * DF_CAND_BYTES;
+    const int b_end = p.b_cand_off + T * DF_CAND_BYTES + (p.b_fb_off < 0 ? 0 : T * p.b_fb_stride);
     *dyn_bytes = 1024 + p.total;
     if (p.a_xp_off + NB * 4 * T * 8 > DF_WARPS * DF_NBUF * DF_CODE_SLOT) return false;
-    if (p.b_off_off + MOE_MAX_E * 4 > DF_WARPS * DF_NBUF * DF_CODE_SLOT) return false;
+    if (b_end > DF_WARPS * DF_NBUF * DF_CODE_SLOT) return false;
     return *dyn_bytes <= max_dyn;
 }
 
@@ -235,6 +258,57 @@ __device__ __forceinline__ void unpack8(uint32_t w, uint32_t (&p)[4]) {
     }
 }
 
+// fp16 pairs of 8 codes for the gate/up MMAs.  The exponent-bias pattern
+// 0x6400 | v is the fp16 value 1024 + v (ulp 1 at 1024), so a code that sits
+// at bit 4 of its field (4-bit: the odd elements; 2-bit: bits 2, 4, 6) gives
+// 1024 + m q with m = 16 (or 4, 16, 64) and needs no shift: one LOP3 per
+// pair.  The matching x fragment holds x' / m, so each product is
+// 1024 x' / m + q x'; the block correction removes the first term and the
+// offset.  4-bit: w = codes 0..7 in nibbles, pairs (0,4) m=1, (1,5) m=16,
+// (2,6) m=1, (3,7) m=16.  2-bit: bytes `sel` (0x4140: bytes 0-1, 0x4342:
+// bytes 2-3) of w hold codes 0..7, pairs (0,4) m=1, (1,5) m=4, (2,6) m=16,
+// (3,7) m=64.
+template <int BITS>
+__device__ __forceinline__ void unpack8_f16(uint32_t w, uint32_t sel, uint32_t (&p)[4]) {
+    constexpr uint32_t kMagic = 0x64006400u;
+    if (BITS == 4) {
+        const uint32_t w8 = w >> 8;
+        p[0] = (w & 0x000F000Fu) | kMagic;
+        p[1] = (w & 0x00F000F0u) | kMagic;
+        p[2] = (w8 & 0x000F000Fu) | kMagic;
+        p[3] = (w8 & 0x00F000F0u) | kMagic;
+    } else {
+        const uint32_t v = __byte_perm(w, 0, sel);  // codes 0-3 in byte 0, codes 4-7 in byte 2
+        p[0] = (v & 0x00030003u) | kMagic;
+        p[1] = (v & 0x000C000Cu) | kMagic;
+        p[2] = (v & 0x00300030u) | kMagic;
+        p[3] = (v & 0x00C000C0u) | kMagic;
+    }
+}
+
+// Factor m of pair i of a gate/up fragment (see unpack8_f16).
+template <int BITS>
+__host__ __device__ constexpr float df_pair_m(int i) {
+    return BITS == 4 ? ((i & 1) ? 16.f : 1.f) : (float)(1 << (2 * i));
+}
+
+// D(4 fp32) = A(16x16 f16) * B(16x8 f16) + C (C a separate register quad).
+__device__ __forceinline__ void mma_f16_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1, const float4& c) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c.x), "f"(c.y), "f"(c.z), "f"(c.w));
+}
+
+// D(4 fp32) += A(16x16 f16) * B(16x8 f16).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // D(4 fp32) += A(16x16 bf16) * B(16x8 bf16).  (Not volatile: a pure function
 // of its operands, which the compiler may schedule freely.)
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -276,16 +350,6 @@ __device__ __forceinline__ void ldsm_x4(const void* row_addr, uint32_t& r0, uint
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(smem_u32(row_addr)));
-}
-
-// 8 bf16 of a row in the fragment order used for B: elements (0,4),(1,5),(2,6),(3,7)
-__device__ __forceinline__ uint4 frag_order8(const float (&v)[8]) {
-    uint4 r;
-    r.x = pack_bf16x2(v[0], v[4]);
-    r.y = pack_bf16x2(v[1], v[5]);
-    r.z = pack_bf16x2(v[2], v[6]);
-    r.w = pack_bf16x2(v[3], v[7]);
-    return r;
 }
 
 // Position of element i (0..I) of a row of h in the fragment order.
@@ -331,10 +395,6 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
@@ -357,65 +417,73 @@ struct DfRoute {  // grouping of the window's pairs, identical in every CTA; arr
 
 // ---------------------------------------------------------------- phase B: top-k of one token
 
-// The selection of topk_token<2> with a shorter first step.  Lanes hold
-// experts e = lane + 32 i, read as (logit, error bound) records.  Every entry
-// at or above theta, the M-th largest of the 32 lane maxima, is a candidate:
-// at least M entries (the lane maxima themselves) reach theta, so the
-// candidates contain the M largest.  With at most 32 of them they are
-// compacted one per lane, sorted by (logit desc, expert asc) and certified as
-// in topk_token; otherwise, or when the certification fails, topk_token<2>
-// decides from scratch (its exact fallback included).  Loops are unrolled so
-// that the shuffles of one step overlap.
-__device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* rec, int t, int32_t* idx_out,
-                                              float* w_out, int* cs, double* cvs, int32_t* nrechk) {
+// Order-preserving integer keys of a logit: key32 of its fp32 rounding (for
+// the coarse candidate step) and key64 of the fp64 value itself (an exact
+// total order, equal values equal keys).  Both are ALU work: on this part a
+// chain of fp64 compares and maxima costs several times more latency.
+__device__ __forceinline__ uint32_t df_key32(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ unsigned long long df_key64(double d) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(d);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// The selection of topk_token<2> with a shorter first step.  Lanes read the
+// (logit, error bound) records of experts e = lane + 32 i from this CTA's
+// shared-memory copy.  Every entry whose fp32 key is at or above theta, the
+// M-th largest of the 32 lane-maximum keys, is a candidate: at least M entries
+// (the lane maxima themselves) reach theta, so the candidates contain the M
+// largest in fp32, and every entry left out is below them by the fp32 rounding
+// at most - the certification below uses the exact upper end of everything
+// left out (rounded up to fp32), so a candidate set that misses a member of the
+// true top k only fails it.  With at most 32 candidates they are sorted by
+// (exact fp64 value desc, expert asc), one per lane, and certified as in
+// topk_token; otherwise, or when the certification fails, topk_token<2>
+// decides from scratch (its exact fallback included).
+__device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* rec, const uint2* reck, int t,
+                                              int32_t* idx_out, float* w_out, int* cs, double* cvs, int* fcs,
+                                              double* fcvs, int32_t* nrechk) {
     const int lane = threadIdx.x & 31;
     const int E = a.E, k = a.k;
-    constexpr int NV = MOE_MAX_E / 32;
-    double v[NV], dl[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int e = lane + 32 * i;
-        double2 r = make_double2(-INFINITY, 0.0);
-        if (e < E) r = __ldcg(rec + e);
-        v[i] = order_val(r.x);
-        dl[i] = order_bnd(r.y);
-    }
     const int M = min(min(E, k + MOE_CAND_EXTRA), 32);
-    double m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) m = fmax(m, v[i]);
-    int r = 0;  // rank of this lane's maximum (descending, ties by lane)
+    uint32_t km = 0;  // this lane's largest key (invalid entries: key 0)
 #pragma unroll 4
+    for (int e = lane; e < E; e += 32) km = max(km, reck[e].x);
+    int r = 0;  // rank of this lane's maximum (descending, ties by lane)
+#pragma unroll 8
     for (int j = 0; j < 32; ++j) {
-        const double o = __shfl_sync(0xffffffffu, m, j);
-        r += (o > m || (o == m && j < lane)) ? 1 : 0;
+        const uint32_t o = __shfl_sync(0xffffffffu, km, j);
+        r += (o > km || (o == km && j < lane)) ? 1 : 0;
     }
-    const unsigned sel = __ballot_sync(0xffffffffu, r == M - 1);
-    const double th = __shfl_sync(0xffffffffu, m, __ffs(sel) - 1);
-    unsigned bm[NV];
-    double rest = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const bool valid = lane + 32 * i < E;
-        const bool in = valid && v[i] >= th;
-        bm[i] = __ballot_sync(0xffffffffu, in);
-        if (valid && !in) rest = fmax(rest, hi_end(v[i], dl[i]));
-    }
+    const uint32_t thk = __shfl_sync(0xffffffffu, km, __ffs(__ballot_sync(0xffffffffu, r == M - 1)) - 1);
+    DF_MARK(20);
     int nc = 0;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        if ((bm[i] >> lane) & 1u) {
-            const int pos = nc + __popc(bm[i] & ((1u << lane) - 1));
+    float rest = -INFINITY;  // an upper end of everything that is not a candidate
+#pragma unroll 4
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const uint2 q = e < E ? reck[e] : make_uint2(0u, __float_as_uint(-INFINITY));
+        const bool in = e < E && q.x >= thk;
+        const unsigned bm = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const int pos = nc + __popc(bm & ((1u << lane) - 1));
             if (pos < 32) {
-                cs[pos] = lane + 32 * i;
-                cvs[pos] = v[i];
-                cvs[32 + pos] = dl[i];
+                const double2 r2 = rec[e];
+                cs[pos] = e;
+                cvs[pos] = r2.x;
+                cvs[32 + pos] = r2.y;
             }
+        } else {
+            rest = fmaxf(rest, __uint_as_float(q.y));  // the upper end, rounded up to fp32
         }
-        nc += __popc(bm[i]);
+        nc += __popc(bm);
     }
-    rest = warp_max_d(rest);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rest = fmaxf(rest, __shfl_xor_sync(0xffffffffu, rest, o));
     __syncwarp();
+    DF_MARK(21);
     if (nc <= 32) {
         double cval = -INFINITY, cbnd = 0.0;
         int ce = 0x7fffffff;
@@ -424,13 +492,16 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
             cbnd = cvs[32 + lane];
             ce = cs[lane];
         }
-        // position of this candidate in (value desc, expert asc) order
+        // position of this candidate in (value desc, expert asc) order, on exact integer keys
+        const unsigned long long ck = lane < nc ? df_key64(cval) : 0ull;
+        const uint32_t ckh = (uint32_t)(ck >> 32), ckl = (uint32_t)ck;
         int rank = 0;
-#pragma unroll 4
+#pragma unroll 8
         for (int j = 0; j < 32; ++j) {
-            const double oj = __shfl_sync(0xffffffffu, cval, j);
+            const uint32_t oh = __shfl_sync(0xffffffffu, ckh, j), ol = __shfl_sync(0xffffffffu, ckl, j);
             const int ej = __shfl_sync(0xffffffffu, ce, j);
-            rank += (j < nc && (oj > cval || (oj == cval && ej < ce))) ? 1 : 0;
+            const unsigned long long ok2 = ((unsigned long long)oh << 32) | ol;
+            rank += (j < nc && (ok2 > ck || (ok2 == ck && ej < ce))) ? 1 : 0;
         }
         __syncwarp();
         if (lane < nc) {  // scatter into sorted order through the scratch
@@ -444,29 +515,16 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
             cbnd = cvs[32 + lane];
             ce = cs[lane];
         }
-        const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
-        const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
-        bool ok = true;
-        if (lane < k && lane + 1 < nc) ok = lo_end(cval, cbnd) > hi_end(nv, nb);
-        if (lane == k - 1) ok = ok && (rest == -INFINITY || lo_end(cval, cbnd) > rest);
-        if (__all_sync(0xffffffffu, ok)) {
+        const bool ok = certify_sorted(cval, cbnd, nc, k, (double)rest);
+        DF_MARK(22);
+        if (ok) {
             write_topk(k, cval, ce, idx_out, w_out);
             return;
         }
     }
     __syncwarp();
-    topk_token<2>(a, t, idx_out, w_out, cs, cvs, nrechk);
-}
-
-// ---------------------------------------------------------------- L2 prefetch of a selected expert
-
-// This CTA's 1/G slice [lo, lo + n) of expert slot `sl`, prefetched into L2.
-// Every CTA issues its slice of each selected expert as soon as a token's
-// selection is known, so the window's expert bytes start streaming from HBM
-// before the grouping is built and the first unit is requested; the units'
-// own loads then find them in L2 (or already in flight).
-__device__ __forceinline__ void df_prefetch_slot(const DecodeFusedArgs& a, int sl, uint32_t lo, uint32_t n) {
-    if (n > 0) prefetch_l2(a.arena + (int64_t)sl * a.slot_bytes + lo, n);
+    DF_MARK(23);
+    topk_token<2>(a, t, idx_out, w_out, fcs, fcvs, nrechk);
 }
 
 // ---------------------------------------------------------------- phase C: one gate/up unit
@@ -519,8 +577,10 @@ __device__ __forceinline__ float df_scale(const uint4* s, int j) {
 }
 
 // accg / accu (rows g, g + 8; token columns 2q, 2q + 1) += the unit's blocks
-// J0 .. J0 + NB - 1.  xb: x fragments [H/32][4][T]; xc: per (block, lane q)
-// the MMA's C quad (c_2q, c_2q+1, c_2q, c_2q+1), c = -(128 + offset) sum x.
+// J0 .. J0 + NB - 1, in units of the scaled x'.  xb: fp16 x fragments
+// [H/32][4][T] (x' / m, see unpack8_f16); xc: per (block, lane q) the MMA's C
+// quad (c_2q, c_2q+1, c_2q, c_2q+1), c = -sum over the block of
+// (1024 + offset m) x' / m.
 template <int BITS>
 __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4* xb, const float4* xc, int J0, int T,
                                              float (&accg)[4], float (&accu)[4]) {
@@ -532,18 +592,18 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
         uint4 bx = make_uint4(0u, 0u, 0u, 0u);
         if (g < T) bx = xb[(J * 4 + q) * T + g];
         const float4 c = xc[J * 4 + q];
-        const int sh = BITS == 2 ? 16 * (j & 1) : 0;
+        const uint32_t sel = (j & 1) ? 0x4342u : 0x4140u;  // 2-bit: the block's half of the word
         const int wi = BITS == 2 ? (j >> 1) : j;
         uint32_t pg0[4], pg1[4], pu0[4], pu1[4];
-        unpack8<BITS>(r.g0[wi] >> sh, pg0);
-        unpack8<BITS>(r.g1[wi] >> sh, pg1);
-        unpack8<BITS>(r.u0[wi] >> sh, pu0);
-        unpack8<BITS>(r.u1[wi] >> sh, pu1);
+        unpack8_f16<BITS>(r.g0[wi], sel, pg0);
+        unpack8_f16<BITS>(r.g1[wi], sel, pg1);
+        unpack8_f16<BITS>(r.u0[wi], sel, pu0);
+        unpack8_f16<BITS>(r.u1[wi], sel, pu1);
         float dg[4], du[4];
-        mma_bf16_16816_c(dg, pg0[0], pg1[0], pg0[1], pg1[1], bx.x, bx.y, c);
-        mma_bf16_16816_c(du, pu0[0], pu1[0], pu0[1], pu1[1], bx.x, bx.y, c);
-        mma_bf16_16816(dg, pg0[2], pg1[2], pg0[3], pg1[3], bx.z, bx.w);
-        mma_bf16_16816(du, pu0[2], pu1[2], pu0[3], pu1[3], bx.z, bx.w);
+        mma_f16_16816_c(dg, pg0[0], pg1[0], pg0[1], pg1[1], bx.x, bx.y, c);
+        mma_f16_16816_c(du, pu0[0], pu1[0], pu0[1], pu1[1], bx.x, bx.y, c);
+        mma_f16_16816(dg, pg0[2], pg1[2], pg0[3], pg1[3], bx.z, bx.w);
+        mma_f16_16816(du, pu0[2], pu1[2], pu0[3], pu1[3], bx.z, bx.w);
         const float sg0 = df_scale(r.sg0, j), sg1 = df_scale(r.sg1, j);
         const float su0 = df_scale(r.su0, j), su1 = df_scale(r.su1, j);
         accg[0] = fmaf(sg0, dg[0], accg[0]);
@@ -615,41 +675,65 @@ __device__ __forceinline__ void df_compute_d_smem(const uint8_t* code, const uin
 
 // ---------------------------------------------------------------- the kernel
 
+// Device-side pointers into the shared-memory plan, common to both kernels.
+struct DfSmem {
+    uint8_t* base;
+    uint8_t* ring;
+    DfRoute rt;
+    uint64_t* full;  // [DF_WARPS][DF_NBUF] unit slots
+    uint64_t* abar;  // x rows (and the slot-table row); records
+    uint64_t* wbar;  // W_r rows
+    int32_t* stab;
+};
+
+__device__ __forceinline__ DfSmem df_smem(uint8_t* smem_raw, const DfPlan& pl, int P) {
+    DfSmem m;
+    // 1024-byte aligned base, derived by pointer arithmetic so that every access
+    // through it compiles to a shared-memory (not generic) load or store
+    m.base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    m.ring = m.base;
+    m.rt.idx = reinterpret_cast<int32_t*>(m.base + pl.route_off);
+    m.rt.w = reinterpret_cast<float*>(m.rt.idx + P);
+    m.rt.perm = reinterpret_cast<int32_t*>(m.rt.w + P);
+    m.rt.inv = m.rt.perm + P;
+    m.rt.u_e = m.rt.inv + P;
+    m.rt.u_pos = m.rt.u_e + P;
+    m.rt.u_n = m.rt.u_pos + P;
+    m.rt.u_sl = m.rt.u_n + P;
+    m.rt.n_uniq = m.rt.u_sl + P;
+    m.full = reinterpret_cast<uint64_t*>(m.base + pl.bar_off);
+    m.abar = m.full + DF_WARPS * DF_NBUF;
+    m.wbar = m.abar + 1;
+    m.stab = reinterpret_cast<int32_t*>(m.base + pl.stab_off);
+    return m;
+}
+
+// ---------------------------------------------------------------- the kernel
+
 template <int BGU, int BD, int NBD>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     k_decode_fused(const __grid_constant__ CUtensorMap tgu, const __grid_constant__ CUtensorMap tcd,
                    DecodeFusedArgs a) {
     extern __shared__ uint8_t smem_raw[];
     constexpr int CK = df_ck(BGU), NBU = CK / 32;  // codes and quant blocks per gate/up unit
-    // 1024-byte aligned base, derived by pointer arithmetic so that every access
-    // through it compiles to a shared-memory (not generic) load or store
-    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const DfPlan& pl = a.pl;
     const int H = a.H, I = a.I, E = a.E, k = a.k, T = a.T, P = T * k, NB = H / 32;
-    uint8_t* ring = base;               // code slots [warp][DF_NBUF][DF_CODE_SLOT]
+    DfSmem sm = df_smem(smem_raw, pl, P);
+    uint8_t* base = sm.base;
+    uint8_t* ring = sm.ring;            // code slots [warp][DF_NBUF][DF_CODE_SLOT]
     uint8_t* scr = base + pl.sc_off;    // scale slots [warp][DF_NBUF][sc_slot]
     uint4* xb = reinterpret_cast<uint4*>(base + pl.r1_off);
     float4* xc = reinterpret_cast<float4*>(base + pl.xc_off);
     float* part = reinterpret_cast<float*>(base + pl.part_off);
-    DfRoute rt;
-    rt.idx = reinterpret_cast<int32_t*>(base + pl.route_off);
-    rt.w = reinterpret_cast<float*>(rt.idx + P);
-    rt.perm = reinterpret_cast<int32_t*>(rt.w + P);
-    rt.inv = rt.perm + P;
-    rt.u_e = rt.inv + P;
-    rt.u_pos = rt.u_e + P;
-    rt.u_n = rt.u_pos + P;
-    rt.u_sl = rt.u_n + P;
-    rt.n_uniq = rt.u_sl + P;
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + pl.bar_off);  // [DF_WARPS][DF_NBUF]
-    uint64_t* abar = full + DF_WARPS * DF_NBUF;  // x rows and the slot-table row
-    uint64_t* wbar = abar + 1;                   // this CTA's W_r rows
-    const int32_t* stab = reinterpret_cast<const int32_t*>(base + pl.stab_off);
-    __shared__ int s_warp[33];
+    DfRoute& rt = sm.rt;
+    uint64_t* full = sm.full;
+    uint64_t* abar = sm.abar;
+    uint64_t* wbar = sm.wbar;
+    const int32_t* stab = sm.stab;
     __shared__ float s_xnorm[DF_TN];
     __shared__ float s_wn[DF_MAX_EPC];
+    __shared__ float s_xsc[DF_TN], s_xinv[DF_TN];  // per token: x' = x * s_xsc, a power of two
     __shared__ int s_ustart[DF_WARPS + 1];  // first gate/up unit of each warp
-
     const int G = gridDim.x, cta = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -676,27 +760,95 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         for (int e = 0; e < ne; ++e) bulk_load(ws + e * wstride, a.W + (size_t)(e0 + e) * H, (uint32_t)(4 * H), wbar);
         mbar_arrive_expect_tx(abar, (uint32_t)(T * 2 * H + E * 4));
         for (int t = 0; t < T; ++t) bulk_load(xs + t * xstride, a.x + (size_t)t * H, (uint32_t)(2 * H), abar);
-        bulk_load(base + pl.stab_off, a.slot_table + (size_t)a.layer * E, (uint32_t)(E * 4), abar);
+        bulk_load(sm.base + pl.stab_off, a.slot_table + (size_t)a.layer * E, (uint32_t)(E * 4), abar);
     }
-    bool alive = mbar_wait(abar, 0, 1, 0);  // the x fragments are built while W_r is still arriving
+    bool alive = mbar_wait(abar, 0, 1, 0);
     DF_MARK(1);
-    // x as MMA B fragments [H/32][4][T], its block sums and squares
-    float* xp = reinterpret_cast<float*>(ring + pl.a_xp_off);  // [2][H/32][4][T]
-    const int nxf = NB * 4 * T;
-    for (int u = tid; u < nxf; u += DF_THREADS) {
-        const int n = u % T, q = (u / T) % 4, j = u / (4 * T);
-        const uint4 r4 = *reinterpret_cast<const uint4*>(xs + n * xstride + (32 * j + 8 * q) * 2);
-        float v[8];
-        v[0] = __uint_as_float(r4.x << 16); v[1] = __uint_as_float(r4.x & 0xffff0000u);
-        v[2] = __uint_as_float(r4.y << 16); v[3] = __uint_as_float(r4.y & 0xffff0000u);
-        v[4] = __uint_as_float(r4.z << 16); v[5] = __uint_as_float(r4.z & 0xffff0000u);
-        v[6] = __uint_as_float(r4.w << 16); v[7] = __uint_as_float(r4.w & 0xffff0000u);
-        xb[u] = frag_order8(v);
-        xp[u] = ((((((v[0] + v[1]) + v[2]) + v[3]) + v[4]) + v[5]) + v[6]) + v[7];
+    if (warp < T) {  // ||x_t|| for the top-k bounds (inflated over its fp32 rounding), while W_r arrives
         float sq = 0.f;
+        for (int i = lane * 8; i < H; i += 256) {
+            const uint4 r4 = *reinterpret_cast<const uint4*>(xs + warp * xstride + i * 2);
+            const uint32_t wd[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
-        for (int z = 0; z < 8; ++z) sq = fmaf(v[z], v[z], sq);
-        xp[nxf + u] = sq;
+            for (int z = 0; z < 4; ++z) {
+                const float lo = __uint_as_float(wd[z] << 16), hi = __uint_as_float(wd[z] & 0xffff0000u);
+                sq = fmaf(lo, lo, fmaf(hi, hi, sq));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) s_xnorm[warp] = sqrtf(sq) * 1.001f;
+    }
+    // x as fp16 MMA fragments, built while the W_r rows arrive
+    {
+        const int xstride = 2 * H + 16;
+        const uint8_t* xs = ring;
+        if (warp < T) {  // per token a power of two that puts max |x| in [2^13, 2^14): the fp16 range holds x'
+            float m = 0.f;
+            for (int i = lane * 8; i < H; i += 256) {
+                const uint4 r4 = *reinterpret_cast<const uint4*>(xs + warp * xstride + i * 2);
+                const uint32_t wd[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+                for (int z = 0; z < 4; ++z)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wd[z] << 16)), fabsf(__uint_as_float(wd[z] & 0xffff0000u))));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) {
+                int ex = 0;
+                const bool fin = m > 0.f && m <= 3.0e38f;  // zero or non-finite rows keep scale 1
+                if (fin) frexpf(m, &ex);                    // m in [2^(ex-1), 2^ex)
+                const int sh = fin ? 14 - ex : 0;
+                s_xsc[warp] = ldexpf(1.f, sh);
+                s_xinv[warp] = ldexpf(1.f, -sh);
+            }
+        } else if (warp < DF_TN && lane == 0) {
+            s_xsc[warp] = 1.f;
+            s_xinv[warp] = 1.f;
+        }
+        __syncthreads();
+        // x as fp16 MMA B fragments [H/32][4][T] (x' / m per pair, see unpack8_f16)
+        // and the block-correction parts
+        float* xp = reinterpret_cast<float*>(ring + pl.a_xp_off);  // [H/32][4][T]
+        const int nxf = NB * 4 * T;
+        constexpr float kOffGU = (float)(1 << (BGU - 1));
+        for (int u = tid; u < nxf; u += DF_THREADS) {
+            const int n = u % T, q = (u / T) % 4, j = u / (4 * T);
+            const uint4 r4 = *reinterpret_cast<const uint4*>(xs + n * xstride + (32 * j + 8 * q) * 2);
+            float v[8];
+            v[0] = __uint_as_float(r4.x << 16); v[1] = __uint_as_float(r4.x & 0xffff0000u);
+            v[2] = __uint_as_float(r4.y << 16); v[3] = __uint_as_float(r4.y & 0xffff0000u);
+            v[4] = __uint_as_float(r4.z << 16); v[5] = __uint_as_float(r4.z & 0xffff0000u);
+            v[6] = __uint_as_float(r4.w << 16); v[7] = __uint_as_float(r4.w & 0xffff0000u);
+            const float sc = s_xsc[n];
+            uint32_t fr[4];
+            float cs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // pair i = elements (i, i + 4), factor m
+                const float im = 1.f / df_pair_m<BGU>(i);  // exact: a power of two
+                const __half2 hv = __floats2half2_rn(v[i] * sc * im, v[i + 4] * sc * im);
+                fr[i] = *reinterpret_cast<const uint32_t*>(&hv);
+                const float2 bb = __half22float2(hv);
+                cs += (1024.f + kOffGU * df_pair_m<BGU>(i)) * (bb.x + bb.y);  // exact products, rounded sum
+            }
+            xb[u] = make_uint4(fr[0], fr[1], fr[2], fr[3]);
+            xp[u] = cs;
+        }
+        __syncthreads();
+        for (int u = tid; u < NB * 4; u += DF_THREADS) {  // block corrections as MMA C quads, zero beyond T
+            const int q = u % 4, j = u / 4;
+            float sx[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                const int n = 2 * q + z;
+                sx[z] = 0.f;
+                if (n < T) {
+                    const float* pp = xp + (size_t)j * 4 * T + n;
+                    sx[z] = ((pp[0] + pp[T]) + pp[2 * T]) + pp[3 * T];
+                }
+            }
+            xc[u] = make_float4(-sx[0], -sx[1], -sx[0], -sx[1]);
+        }
     }
     alive = mbar_wait(wbar, 0, 1, 1) && alive;
     DF_MARK(2);
@@ -706,67 +858,59 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         const bool erow = g < ne, xrow_ok = g < T;
         const uint8_t* wrow = ws + (erow ? g : 0) * wstride;
         const uint8_t* xrow = xs + (xrow_ok ? g : 0) * xstride;
-        double c0 = 0.0, c1 = 0.0;
+        // two accumulator chains (even and odd 16-element slices) halve the dependent MMA chain
+        double c0 = 0.0, c1 = 0.0, d0 = 0.0, d1 = 0.0;
         float w2 = 0.f;
-#pragma unroll 4
-        for (int k0 = kb; k0 < kb + kw; k0 += 16) {
-            // step s of this 16-element slice uses k = k0 + 4 q + s (A and B alike)
-            const float4 wv = erow ? *reinterpret_cast<const float4*>(wrow + (k0 + 4 * q) * 4) : make_float4(0, 0, 0, 0);
-            const uint2 xv = xrow_ok ? *reinterpret_cast<const uint2*>(xrow + (k0 + 4 * q) * 2) : make_uint2(0, 0);
-            w2 = fmaf(wv.x, wv.x, fmaf(wv.y, wv.y, fmaf(wv.z, wv.z, fmaf(wv.w, wv.w, w2))));
-            const double av[4] = {wv.x, wv.y, wv.z, wv.w};
-            const double bv[4] = {__uint_as_float(xv.x << 16), __uint_as_float(xv.x & 0xffff0000u),
-                                  __uint_as_float(xv.y << 16), __uint_as_float(xv.y & 0xffff0000u)};
+#pragma unroll 2
+        for (int k0 = kb; k0 < kb + kw; k0 += 32) {
 #pragma unroll
-            for (int st = 0; st < 4; ++st)
-                asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-                             : "+d"(c0), "+d"(c1)
-                             : "d"(av[st]), "d"(bv[st]));
+            for (int half = 0; half < 2; ++half) {
+                // step s of this 16-element slice uses k = k1 + 4 q + s (A and B alike)
+                const int k1 = k0 + 16 * half;
+                const float4 wv = erow ? *reinterpret_cast<const float4*>(wrow + (k1 + 4 * q) * 4) : make_float4(0, 0, 0, 0);
+                const uint2 xv = xrow_ok ? *reinterpret_cast<const uint2*>(xrow + (k1 + 4 * q) * 2) : make_uint2(0, 0);
+                w2 = fmaf(wv.x, wv.x, fmaf(wv.y, wv.y, fmaf(wv.z, wv.z, fmaf(wv.w, wv.w, w2))));
+                const double av[4] = {wv.x, wv.y, wv.z, wv.w};
+                const double bv[4] = {__uint_as_float(xv.x << 16), __uint_as_float(xv.x & 0xffff0000u),
+                                      __uint_as_float(xv.y << 16), __uint_as_float(xv.y & 0xffff0000u)};
+#pragma unroll
+                for (int st = 0; st < 4; ++st) {
+                    if (half == 0)
+                        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                                     : "+d"(c0), "+d"(c1)
+                                     : "d"(av[st]), "d"(bv[st]));
+                    else
+                        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                                     : "+d"(d0), "+d"(d1)
+                                     : "d"(av[st]), "d"(bv[st]));
+                }
+            }
         }
-        // c0, c1: expert e0 + g, tokens 2q, 2q+1 (this warp's slice of H)
+        // expert e0 + g, tokens 2q, 2q+1 (this warp's slice of H)
         double* sp = reinterpret_cast<double*>(ring + pl.a_sp_off);
-        sp[(warp * 8 + g) * 8 + 2 * q] = c0;
-        sp[(warp * 8 + g) * 8 + 2 * q + 1] = c1;
+        sp[(warp * 8 + g) * 8 + 2 * q] = c0 + d0;
+        sp[(warp * 8 + g) * 8 + 2 * q + 1] = c1 + d1;
         w2 += __shfl_xor_sync(0xffffffffu, w2, 1);
         w2 += __shfl_xor_sync(0xffffffffu, w2, 2);
         float* sw2 = reinterpret_cast<float*>(ring + pl.a_w2_off);
         if (q == 0) sw2[warp * 8 + g] = w2;
     }
     __syncthreads();
-    if (warp < T) {  // ||x_t|| for the top-k bounds (inflated over its fp32 rounding)
-        float sq = 0.f;
-        for (int u = lane; u < NB * 4; u += 32) sq += xp[nxf + u * T + warp];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        if (lane == 0) s_xnorm[warp] = sqrtf(sq) * 1.001f;
-    } else if (warp == T && lane < ne) {  // ||W_r[e]|| of this CTA's experts
+    if (warp == 0 && lane < ne) {  // ||W_r[e]|| of this CTA's experts
         const float* sw2 = reinterpret_cast<const float*>(ring + pl.a_w2_off);
         float s2 = 0.f;
         for (int w = 0; w < DF_WARPS; ++w) s2 += sw2[w * 8 + lane];
         s_wn[lane] = sqrtf(s2) * 1.001f;
         a.wnorm[e0 + lane] = s_wn[lane];
     }
-    for (int u = tid; u < NB * 4; u += DF_THREADS) {  // block corrections as MMA C quads, zero beyond T
-        const int q = u % 4, j = u / 4;
-        float sx[2];
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-            const int n = 2 * q + z;
-            sx[z] = 0.f;
-            if (n < T) {
-                const float* pp = xp + (size_t)j * 4 * T + n;
-                sx[z] = ((pp[0] + pp[T]) + pp[2 * T]) + pp[3 * T];
-            }
-        }
-        const float f = -(128.f + (float)(1 << (BGU - 1)));
-        xc[u] = make_float4(f * sx[0], f * sx[1], f * sx[0], f * sx[1]);
-    }
     __syncthreads();
     if (tid < 64 && (tid >> 3) < ne && (tid & 7) < T) {  // logits and their error bounds
         const double* sp = reinterpret_cast<const double*>(ring + pl.a_sp_off);
         const int gg = tid >> 3, t = tid & 7, e = e0 + gg;
-        double sum = 0.0;
-        for (int w = 0; w < DF_WARPS; ++w) sum += sp[(w * 8 + gg) * 8 + t];
+        double part4[4] = {0.0, 0.0, 0.0, 0.0};  // four short chains: fp64 adds have a long latency here
+#pragma unroll
+        for (int w = 0; w < DF_WARPS; ++w) part4[w & 3] += sp[(w * 8 + gg) * 8 + t];
+        const double sum = (part4[0] + part4[1]) + (part4[2] + part4[3]);
         const double bb = a.b ? (double)a.b[e] : 0.0;
         const double lg = sum + bb;
         a.logit[(size_t)t * E + e] = lg;
@@ -774,9 +918,15 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         // sums, H + 2 in the definition's own sequential sum
         const double gam = ((double)(H + 32) + (double)(H + 2)) * 1.1102230246251565e-16 * 1.01;
         const double B = ((double)s_xnorm[t] * (double)s_wn[gg] + fabs(bb)) * 1.001;
-        const double2 r = make_double2(lg, B * gam + 1e-300);
+        const double lv = order_val(lg), bnd = order_bnd(B * gam + 1e-300);
+        const double2 r = make_double2(lv, bnd);
+        // what the candidate step of the top-k needs, in integer / fp32 form
+        const uint2 rk = make_uint2(df_key32((float)lv), __float_as_uint(__double2float_ru(hi_end(lv, bnd))));
 #pragma unroll
-        for (int c = 0; c < DF_NREP; ++c) a.rec[((size_t)c * T + t) * E + e] = r;
+        for (int c = 0; c < DF_NREP; ++c) {
+            a.rec[((size_t)c * T + t) * E + e] = r;
+            a.reck[((size_t)c * T + t) * E + e] = rk;
+        }
     }
     DF_MARK(3);
     {
@@ -785,82 +935,131 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     }
     DF_MARK(4);
 
-    // ---- B: certified top-k of every token (same result in every CTA) and grouping
-    const uint32_t pf_step = (uint32_t)((a.slot_bytes / G + 15) & ~(int64_t)15);
-    const uint32_t pf_lo = pf_step * (uint32_t)cta;
-    const uint32_t pf_n = pf_lo >= a.slot_bytes ? 0u : (uint32_t)min((int64_t)pf_step, a.slot_bytes - pf_lo);
+    // ---- B: certified top-k of every token (the same result in every CTA) and grouping
     if (alive) {
+        // this CTA's copy of the records: one bulk copy into the ring, which
+        // phase A no longer uses (the grid barrier ended its reads)
+        double2* srec = reinterpret_cast<double2*>(ring + pl.b_rec_off);
+        uint2* sreck = reinterpret_cast<uint2*>(ring + pl.b_key_off);
+        if (tid == 0) {
+            fence_proxy_async_global();  // other CTAs wrote the records with plain stores
+            fence_proxy_async_smem();    // and this CTA used the ring through the generic proxy
+            const uint32_t bytes = (uint32_t)(T * E * 16), kbytes = (uint32_t)(T * E * 8);
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(a.rec + (size_t)(cta % DF_NREP) * T * E);
+            const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(a.reck + (size_t)(cta % DF_NREP) * T * E);
+            mbar_arrive_expect_tx(abar, bytes + kbytes);
+            for (uint32_t o = 0; o < bytes; o += 16384)
+                bulk_load(reinterpret_cast<uint8_t*>(srec) + o, src + o, min(16384u, bytes - o), abar);
+            for (uint32_t o = 0; o < kbytes; o += 16384)
+                bulk_load(reinterpret_cast<uint8_t*>(sreck) + o, ksrc + o, min(16384u, kbytes - o), abar);
+        }
+        alive = mbar_wait(abar, 1, 3, 0);
+        DF_MARK(17);
         if (warp < T) {
             TopkArgs ta{};
             ta.x = a.x; ta.W = a.W; ta.b = a.b; ta.logit = a.logit; ta.wnorm = a.wnorm; ta.xnorm = s_xnorm;
             // phase-A sums: at most H + 32 roundings along any product's path
             ta.gfast = (double)(H + 32) * 1.1102230246251565e-16 * 1.01;
             ta.T = T; ta.H = H; ta.E = E; ta.k = k;
-            int* cs = reinterpret_cast<int*>(ring + warp * MOE_MAX_E * 12);  // the ring is free during B
-            double* cvs = reinterpret_cast<double*>(ring + warp * MOE_MAX_E * 12 + MOE_MAX_E * 4);
-            const double2* rec = a.rec + ((size_t)(cta % DF_NREP) * T + warp) * E;
-            df_topk_token(ta, rec, warp, rt.idx + warp * k, rt.w + warp * k, cs, cvs, cta == 0 ? a.nrechk : nullptr);
+            // candidate scratch of this token; the exact fallback reuses the token's own
+            // record row (read by the fast step by then) when it holds max(E,32) ints and
+            // max(E,64) doubles, else its own region
+            int* cs = reinterpret_cast<int*>(ring + pl.b_cand_off + warp * DF_CAND_BYTES);
+            double* cvs = reinterpret_cast<double*>(cs + 32);
+            int* fcs = pl.b_fb_off < 0 ? reinterpret_cast<int*>(srec + (size_t)warp * E)
+                                       : reinterpret_cast<int*>(ring + pl.b_fb_off + warp * pl.b_fb_stride);
+            double* fcvs = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(fcs) + df_al(4 * max(E, 32), 8));
+            if (alive)
+                df_topk_token(ta, srec + (size_t)warp * E, sreck + (size_t)warp * E, warp, rt.idx + warp * k,
+                              rt.w + warp * k, cs, cvs, fcs, fcvs, cta == 0 ? a.nrechk : nullptr);
+            if (warp == 0) DF_MARK(18);
             __syncwarp();
-            if (lane < k) {  // this token's experts start streaming into L2
+            if (alive && lane < k) {
                 const int e = rt.idx[warp * k + lane];
-                const int64_t sl = (unsigned)e < (unsigned)E ? stab[e] : -1;
-                if (sl >= 0 && sl < a.n_slots) df_prefetch_slot(a, (int)sl, pf_lo, pf_n);
+                if ((unsigned)e >= (unsigned)E) {  // never produced by the top-k; a guard against a library fault
+                    rt.idx[warp * k + lane] = 0;
+                    moe_set_status(MOE_ERR_RANGE);
+                }
             }
         }
-        int* s_cnt = reinterpret_cast<int*>(ring + pl.b_cnt_off);
-        int* s_off = reinterpret_cast<int*>(ring + pl.b_off_off);
-        for (int e = tid; e < MOE_MAX_E; e += DF_THREADS) s_cnt[e] = 0;
-        __syncthreads();
+        alive = __syncthreads_and(alive) != 0;
         DF_MARK(5);
-        for (int p = tid; p < P; p += DF_THREADS) {
-            int e = rt.idx[p];
-            if ((unsigned)e >= (unsigned)E) {  // never produced by the top-k; a guard against a library fault
-                e = 0;
-                rt.idx[p] = 0;
-                moe_set_status(MOE_ERR_RANGE);
+    }
+    if (alive) {
+        // grouping: one warp sorts the pairs by (expert, pair id) and lists the
+        // experts; in CTA 0 the other warps count the routing outputs directly
+        if (warp == 0) {
+            int* se = rt.u_n;  // the experts in sorted order (u_n is written after it is read)
+            if (P <= 64) {  // keys e * 64 + p, one or two per lane, ranked with shuffles
+                const int k0 = lane < P ? rt.idx[lane] * 64 + lane : 0x7fffffff;
+                const int k1 = lane + 32 < P ? rt.idx[lane + 32] * 64 + lane + 32 : 0x7fffffff;
+                int r0 = 0, r1 = 0;
+#pragma unroll 8
+                for (int j = 0; j < 32; ++j) {
+                    const int o0 = __shfl_sync(0xffffffffu, k0, j), o1 = __shfl_sync(0xffffffffu, k1, j);
+                    r0 += (o0 < k0 ? 1 : 0) + (o1 < k0 ? 1 : 0);
+                    r1 += (o0 < k1 ? 1 : 0) + (o1 < k1 ? 1 : 0);
+                }
+                if (lane < P) { rt.perm[r0] = lane; rt.inv[lane] = r0; se[r0] = k0 >> 6; }
+                if (lane + 32 < P) { rt.perm[r1] = lane + 32; rt.inv[lane + 32] = r1; se[r1] = k1 >> 6; }
+            } else {
+                for (int p = lane; p < P; p += 32) {
+                    const int e = rt.idx[p];
+                    int r = 0;
+#pragma unroll 8
+                    for (int q2 = 0; q2 < P; ++q2) {
+                        const int f = rt.idx[q2];
+                        r += (f < e || (f == e && q2 < p)) ? 1 : 0;
+                    }
+                    rt.perm[r] = p;
+                    rt.inv[p] = r;
+                    se[r] = e;
+                }
             }
-            atomicAdd(&s_cnt[e], 1);
+            __syncwarp();
+            int nu = 0;
+            for (int r0 = 0; r0 < P; r0 += 32) {
+                const int r = r0 + lane;
+                const int e = r < P ? se[r] : -1;
+                const bool first = r < P && (r == 0 || se[r - 1] != e);
+                const unsigned m = __ballot_sync(0xffffffffu, first);
+                if (first) {
+                    const int u = nu + __popc(m & ((1u << lane) - 1));
+                    const int64_t sl = stab[e];
+                    rt.u_e[u] = e;
+                    rt.u_pos[u] = r;
+                    rt.u_sl[u] = (sl >= 0 && sl < a.n_slots) ? (int32_t)sl : -1;
+                    if (cta == 0 && rt.u_sl[u] < 0) moe_set_status(MOE_ERR_SLOT);
+                }
+                nu += __popc(m);
+            }
+            __syncwarp();
+            for (int u = lane; u < nu; u += 32) rt.u_n[u] = (u + 1 < nu ? rt.u_pos[u + 1] : P) - rt.u_pos[u];
+            if (lane == 0) *rt.n_uniq = nu;
+            DF_MARK(19);
+        } else if (cta == 0) {
+            for (int e = tid - 32; e <= E; e += DF_THREADS - 32) {  // offsets[e] = pairs on experts below e
+                int lt = 0, eq = 0;
+#pragma unroll 8
+                for (int q2 = 0; q2 < P; ++q2) {
+                    const int f = rt.idx[q2];
+                    lt += f < e ? 1 : 0;
+                    eq += f == e ? 1 : 0;
+                }
+                a.offsets[e] = lt;
+                if (e < E && a.hist) a.hist[(size_t)a.layer * E + e] += (uint32_t)eq;
+            }
         }
         __syncthreads();
-        const int c = tid < E ? s_cnt[tid] : 0;
-        int off;
-        const int total = block_excl_scan(c, &off, s_warp);
-        if (tid < E) s_off[tid] = off;
-        int upos;
-        const int nu = block_excl_scan((tid < E && c > 0) ? 1 : 0, &upos, s_warp);
-        if (tid < E && c > 0) {
-            const int64_t sl = stab[tid];
-            rt.u_e[upos] = tid;
-            rt.u_pos[upos] = off;
-            rt.u_n[upos] = c;
-            rt.u_sl[upos] = (sl >= 0 && sl < a.n_slots) ? (int32_t)sl : -1;
-            if (cta == 0 && rt.u_sl[upos] < 0) moe_set_status(MOE_ERR_SLOT);
-        }
-        if (tid == 0) *rt.n_uniq = nu;
-        if (cta == 0) {
-            if (tid < E) {
-                a.offsets[tid] = off;
-                if (a.hist) a.hist[(size_t)a.layer * E + tid] += (uint32_t)c;
-            }
-            if (tid == 0) a.offsets[E] = total;
-        }
-        __syncthreads();
-        for (int p = tid; p < P; p += DF_THREADS) {
-            const int e = rt.idx[p];
-            int before = 0;
-            for (int q2 = 0; q2 < p; ++q2) before += (rt.idx[q2] == e);
-            const int pos = s_off[e] + before;
-            rt.perm[pos] = p;
-            rt.inv[p] = pos;
-            if (cta == 0) {
-                a.perm[pos] = p;
-                a.idx[p] = e;
+        if (cta == 0)
+            for (int p = tid; p < P; p += DF_THREADS) {
+                a.perm[p] = rt.perm[p];
+                a.idx[p] = rt.idx[p];
                 a.w[p] = rt.w[p];
             }
-        }
-        __syncthreads();
     }
     DF_MARK(6);
+    DF_CLK(cb0);
 
     // ---- C: gate/up + SwiGLU.  A grid barrier separates C from D, so each phase
     // is balanced on its own: every CTA takes an equal share of the 16-row
@@ -947,6 +1146,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         __syncwarp();
         for (; issued < min(S, DF_NBUF); ++issued) issue(issued);
     }
+    DF_CLK(cl0);
+    if (nC > 0) DF_WACC(9, cl0 - cb0);
     bool wok = true;
     int s = 0;  // units consumed
     {
@@ -954,8 +1155,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         const int g = lane >> 2, q = lane & 3;
         for (; s < nC; ++s) {
             const int b = s % DF_NBUF;
+            DF_CLK(c0);
             if (!mbar_wait(&full[warp * DF_NBUF + b], (uint32_t)(s / DF_NBUF) & 1u, 4, s)) { wok = false; break; }
-            if (s == 0) DF_MARK(7);
+            DF_CLK(c1);
+            DF_WACC(0, c1 - c0);
+            DF_WACC(4, 1);
+            if (s == 0) DF_MARK(10);
             const int u = ub + s, lt = u / NCH, ch = u % NCH, gt = r0 + lt, ui = gt / tiles_e;
             const bool valid = rt.u_sl[ui] >= 0;
             DfCRegs<BGU> cr;
@@ -963,18 +1168,26 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                 df_stage_c<BGU>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT, scr + (warp * DF_NBUF + b) * pl.sc_slot,
                                 cr);
             __syncwarp();  // every lane's reads of the slot are done: it may be refilled
+            DF_CLK(c1a);
+            DF_WACC(8, c1a - c1);
             if (issued < S) issue(issued++);  // re-arm the slot with unit s + DF_NBUF
+            DF_CLK(c1b);
+            DF_WACC(7, c1b - c1a);
             if (valid) df_compute_c<BGU>(cr, xb, xc, ch * NBU, T, accg, accu);
+            DF_CLK(c2);
+            DF_WACC(1, c2 - c1);
+            if (s == 0) DF_WACC(6, c2 - c1);
             if (s == nC - 1 || (u + 1) / NCH != lt) {  // this warp's part of tile lt is complete
                 float* pp = part + (size_t)(lt + warp) * (2 * 16 * T);  // [gate, up][16 rows][T]
 #pragma unroll
                 for (int z = 0; z < 2; ++z) {
                     const int col = 2 * q + z;
-                    if (col < T) {
-                        pp[g * T + col] = accg[z];
-                        pp[(g + 8) * T + col] = accg[2 + z];
-                        pp[16 * T + g * T + col] = accu[z];
-                        pp[16 * T + (g + 8) * T + col] = accu[2 + z];
+                    if (col < T) {  // back from x' to x: an exact power-of-two scaling
+                        const float iv = s_xinv[col];
+                        pp[g * T + col] = accg[z] * iv;
+                        pp[(g + 8) * T + col] = accg[2 + z] * iv;
+                        pp[16 * T + g * T + col] = accu[z] * iv;
+                        pp[16 * T + (g + 8) * T + col] = accu[2 + z] * iv;
                     }
                 }
 #pragma unroll
@@ -983,7 +1196,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         }
     }
     const bool cok = __syncthreads_and(wok && alive) != 0;
-    DF_MARK(8);
+    DF_MARK(11);
     // finish the tiles: sum the partials of the warps that covered each tile (in
     // warp order), SwiGLU, round h to bf16 and store it for every pair of the expert
     if (cok) {
@@ -1005,12 +1218,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             a.hB[(size_t)pos * I + frag_pos(r16 * 16 + row)] = f32_to_bf16_bits(h);
         }
     }
-    DF_MARK(9);
+    DF_MARK(12);
     {
         const bool gb = grid_barrier(a.bar, 2u, 2, a.spin_limit);
         alive = __syncthreads_and(cok && gb) != 0;
     }
-    DF_MARK(10);
+    DF_MARK(13);
 
     // ---- D: down projection of this CTA's feature tiles for every selected
     // expert (warp w takes experts w, w + 16, ...), then the combine.
@@ -1036,13 +1249,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             hsum[it] = sum;
         }
         __syncthreads();
-        DF_MARK(11);
+        DF_MARK(14);
     }
     if (alive) {
         const int g = lane >> 2, q = lane & 3;
         for (; s < S; ++s) {
             const int b = s % DF_NBUF;
+            DF_CLK(c0);
             if (!mbar_wait(&full[warp * DF_NBUF + b], (uint32_t)(s / DF_NBUF) & 1u, 6, s)) { wok = false; break; }
+            DF_CLK(c1);
+            DF_WACC(2, c1 - c0);
+            DF_WACC(5, 1);
             const int d = s - nC, rr = d / ndw, ui = warp + DF_WARPS * (d % ndw);
             const int pos0 = rt.u_pos[ui], n = rt.u_n[ui];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1052,6 +1269,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                                            pl.hs_stride, hsum + (size_t)pos0 * nblk_d, n, acc);
             __syncwarp();  // the slot's reads are done: it may be refilled
             if (issued < S) issue(issued++);
+            DF_CLK(c2);
+            DF_WACC(3, c2 - c1);
 #pragma unroll
             for (int z = 0; z < 2; ++z) {  // y for pair columns 2q, 2q+1 (when they exist), features g, g+8
                 const int jj = 2 * q + z;
@@ -1065,7 +1284,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             }
         }
         alive = __syncthreads_and(wok) != 0;
-        DF_MARK(12);
+        DF_MARK(15);
         if (alive)
             for (int u = tid; u < nftc * T * DF_FT; u += DF_THREADS) {
                 const int rr = u / (T * DF_FT), t = (u / DF_FT) % T, fl = u % DF_FT;
@@ -1080,5 +1299,5 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     // On an error path, wait (bounded) for this warp's copies still in flight
     // before the CTA's shared memory goes away.
     for (int r = s; r < issued; ++r) mbar_wait(&full[warp * DF_NBUF + r % DF_NBUF], (uint32_t)(r / DF_NBUF) & 1u, 8, r);
-    DF_MARK(13);
+    DF_MARK(16);
 }

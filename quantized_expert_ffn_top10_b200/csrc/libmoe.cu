@@ -24,7 +24,7 @@ inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
     size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, wsplit,
-        xn, slow, hout, total;
+        xn, slow, hout, reck, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -54,6 +54,7 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.h = put(P * I * (small ? 4 : 2));  // decode keeps h and Y in fp32, prefill in bf16
     w.y = put(P * H * (small ? 4 : 2));
     w.rec = put(small ? (size_t)DF_NREP * T * E * 16 : 0);  // fused decode: replicated (logit, bound) records
+    w.reck = put(small ? (size_t)DF_NREP * T * E * 8 : 0);  // and their keys
     w.wsplit = put(small ? 0 : (size_t)3 * E * H * 2);        // chunk router: W_r as three bf16 planes
     w.xn = put(small ? 0 : (size_t)T * 4);                     // chunk router: ||x_t|| per token
     w.slow = put(small ? 0 : (size_t)(T + 4) * 4);             // chunk top-k: [count, tokens...] left to the slow pass
@@ -412,6 +413,7 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     a.hB = reinterpret_cast<uint16_t*>(c.ws + L.h);
     a.bar = reinterpret_cast<unsigned int*>(c.ws + L.gbar);
     a.rec = reinterpret_cast<double2*>(c.ws + L.rec);
+    a.reck = reinterpret_cast<uint2*>(c.ws + L.reck);
     a.pl = plan;
     a.spin_limit = g_dbg_spin.load() ? g_dbg_spin.load() : MOE_SPIN_LIMIT;
     a.bar1_extra = g_dbg_bar1.load();
@@ -446,7 +448,7 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
                                                                     c.steer, c.out);
         count(1);
     }
-    for (int i = 1; i < 5; ++i) stage(i, c.st);  // one kernel: the stages collapse onto its end
+    stage(1, c.st);  // one kernel: only its start and end are recorded
     count(1);
     return e == cudaSuccess ? cuda_rc(cudaGetLastError()) : MOE_ERR_CUDA;
 }
@@ -848,6 +850,14 @@ int moe_timeout_site(void* stream) {
 // Measurement builds only: the fused decode kernel's phase timestamps of the last launch.
 int moe_probe_read(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_df_probe, sizeof(g_df_probe)) == cudaSuccess ? 0 : -1;
+}
+int moe_probe_warps(unsigned long long* host, int clear) {
+    if (cudaMemcpyFromSymbol(host, g_df_wprobe, sizeof(g_df_wprobe)) != cudaSuccess) return -1;
+    if (clear) {
+        static unsigned long long zero[160 * DF_WARPS_PROBE * DF_NWP];
+        if (cudaMemcpyToSymbol(g_df_wprobe, zero, sizeof(zero)) != cudaSuccess) return -1;
+    }
+    return 0;
 }
 #endif
 

@@ -237,13 +237,51 @@ __device__ __forceinline__ double logit_fp64_exact(const TopkArgs& a, int t, int
 // receives position r.  Returns whether every decision is certified: each of
 // the first k positions is separated from the next, and position k-1 clears
 // `rest` (the upper end of everything outside the candidates).
+// Exact, order-preserving integer key of a (non-NaN) double: ranking on it is
+// ALU work, where chains of fp64 compares cost several times the latency.
+__device__ __forceinline__ unsigned long long order_key64(double d) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(d);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// The largest upper end among the candidates ranked k .. M-1 (lanes in rank
+// order), rounded up to fp32; -inf when there are none.
+__device__ __forceinline__ double tail_hi_end(double cval, double cbnd, int M, int k) {
+    const int lane = threadIdx.x & 31;
+    const float h = (lane >= k && lane < M) ? __double2float_ru(hi_end(cval, cbnd)) : -INFINITY;
+    const uint32_t u = __float_as_uint(h);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, (u & 0x80000000u) ? ~u : (u | 0x80000000u));
+    return (double)__uint_as_float((m & 0x80000000u) ? (m & 0x7fffffffu) : ~m);
+}
+
+// Lanes hold M candidates in (value desc, expert asc) order; `rest` is an upper
+// end of every expert that is not a candidate (-inf when there is none).  The
+// first k are certified as the exact top k in the exact order when the
+// intervals of ranks j and j + 1 are disjoint for j < k - 1 and the lower end
+// of rank k - 1 is above the upper end of every candidate ranked k or later
+// and above `rest`.
+__device__ __forceinline__ bool certify_sorted(double cval, double cbnd, int M, int k, double rest) {
+    const int lane = threadIdx.x & 31;
+    const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
+    const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
+    const double tail = fmax(rest, tail_hi_end(cval, cbnd, M, k));
+    bool ok = true;
+    if (lane < k - 1) ok = lo_end(cval, cbnd) > hi_end(nv, nb);
+    if (lane == k - 1) ok = lo_end(cval, cbnd) > tail;
+    return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int& ce, int M, int k, double rest) {
     const int lane = threadIdx.x & 31;
+    const unsigned long long ck = order_key64(cval);
+    const uint32_t ckh = (uint32_t)(ck >> 32), ckl = (uint32_t)ck;
     int rank = 0;
-    for (int j = 0; j < M; ++j) {
-        double oj = __shfl_sync(0xffffffffu, cval, j);
-        int ej = __shfl_sync(0xffffffffu, ce, j);
-        if (lane < M && (oj > cval || (oj == cval && ej < ce))) ++rank;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+        const uint32_t oh = __shfl_sync(0xffffffffu, ckh, j), ol = __shfl_sync(0xffffffffu, ckl, j);
+        const int ej = __shfl_sync(0xffffffffu, ce, j);
+        const unsigned long long oj = ((unsigned long long)oh << 32) | ol;
+        if (j < M && lane < M && (oj > ck || (oj == ck && ej < ce))) ++rank;
     }
     int src = 0;
     for (int j = 0; j < M; ++j)
@@ -251,12 +289,7 @@ __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int
     cval = __shfl_sync(0xffffffffu, cval, src);
     cbnd = __shfl_sync(0xffffffffu, cbnd, src);
     ce = __shfl_sync(0xffffffffu, ce, src);
-    const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
-    const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
-    bool ok = true;
-    if (lane < k && lane + 1 < M) ok = lo_end(cval, cbnd) > hi_end(nv, nb);
-    if (lane == k - 1) ok = ok && (rest == -INFINITY || lo_end(cval, cbnd) > rest);
-    return __all_sync(0xffffffffu, ok);
+    return certify_sorted(cval, cbnd, M, k, rest);
 }
 
 __device__ __forceinline__ void write_topk(int k, double cval, int ce, int32_t* idx_out, float* w_out) {
@@ -428,11 +461,13 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             }
         }
     }
-    double rest = -INFINITY;
+    float rest_f = -INFINITY;  // an upper end of everything left out, rounded up to fp32 (a short fp32 chain)
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-        if (!((taken >> i) & 1u)) rest = fmax(rest, hi_end(v[i], dl[i]));
-    rest = warp_max_d(rest);
+        if (!((taken >> i) & 1u)) rest_f = fmaxf(rest_f, __double2float_ru(hi_end(v[i], dl[i])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rest_f = fmaxf(rest_f, __shfl_xor_sync(0xffffffffu, rest_f, o));
+    const double rest = (double)rest_f;
 
     // 2) certified on the fast values?
     if (sort_and_certify(cval, cbnd, ce, MC, k, rest)) {
@@ -452,9 +487,15 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     if (MODE == 0) {
         const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
         const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
+        const double lok = __shfl_sync(0xffffffffu, lo_end(cval, cbnd), k - 1);
+        // overlapping adjacent pairs among the k + 1 best, and candidates further
+        // down whose interval reaches the k-th (which then needs its own value too)
         const bool pairbad = lane < k && lane + 1 < MC && !(lo_end(cval, cbnd) > hi_end(nv, nb));
-        const bool prevbad = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0 && lane > 0;
-        const unsigned need = __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad));
+        const bool tailbad = lane > k && lane < MC && !(lok > hi_end(cval, cbnd));
+        const bool anytail = __any_sync(0xffffffffu, tailbad);
+        const bool prevup = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0;
+        const bool prevbad = (prevup && lane > 0) || (lane == k - 1 && anytail);
+        const unsigned need = __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad || tailbad));
         const int NR = __popc(need);
         for (int base = 0; base < NR; base += 16) {
             int ej[16], lj[16];

@@ -80,7 +80,7 @@ __device__ unsigned long long g_df_wprobe[160][DF_WARPS_PROBE][DF_NWP];
 #define DF_MAX_EPC 8       // router experts per CTA (rows of the fp64 MMA)
 #define DF_MAX_NBD 16      // quant blocks of a W_d row (I <= 512)
 #define DF_SMEM_LIMIT (227 * 1024)
-#define DF_BAR_WORDS (32 * 18)  // grid barrier: 16 group counters, the top counter, the flag
+#define DF_BAR_WORDS 32     // grid barrier: one counter on its own 128-byte line
 #define DF_NREP 8          // copies of the (logit, bound) records that phase B reads
 #define DF_CAND_BYTES 640  // phase-B candidate scratch of one token: 32 experts, 32 values + 32 bounds
 
@@ -126,7 +126,7 @@ struct DecodeFusedArgs {
     double2* rec;            // [DF_NREP][T][E] (logit, error bound): CTA c reads copy c % DF_NREP
     uint2* reck;             // [DF_NREP][T][E] (key32 of the fp32 logit, upper end rounded up to fp32)
     uint16_t* hB;            // [P][I] bf16, MMA-fragment order within each 32-block
-    unsigned int* bar;       // grid barrier counters and flag, DF_BAR_WORDS words (zeroed before launch)
+    unsigned int* bar;       // grid barrier counter, DF_BAR_WORDS words (zeroed before launch)
     unsigned spin_limit;     // polling bound of the grid barriers (MOE_SPIN_LIMIT; lowered only by a test)
     unsigned bar1_extra;     // 0; a test sets it to make grid barrier 1 unsatisfiable
     DfPlan pl;
@@ -205,14 +205,12 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
-// Grid-wide barrier over gridDim.x co-resident CTAs, phase `ph` (1, 2, ...),
-// in two levels so that no counter sees more than ~16 arrivals: CTA c arrives
-// on group counter c % DF_BAR_GROUPS; the last arrival of a group arrives on
-// the top counter; the last arrival there stores the phase to the release
-// flag, which the others poll.  Counters and flag sit on separate 128-byte
-// lines of `bar` (zeroed before launch) and only grow.  Bounded: on expiry the
-// status word gets MOE_ERR_TIMEOUT and every thread of the CTA sees false.
-#define DF_BAR_GROUPS 16
+// Grid-wide barrier over gridDim.x co-resident CTAs, phase `ph` (1, 2, ...):
+// thread 0 of every CTA adds one to the counter bar[0] (zeroed before launch,
+// it only grows) and polls it until it reaches ph * gridDim.x.  One counter
+// costs one atomic round trip plus one polling round trip; 148 arrivals on one
+// L2 line serialise in well under that.  Bounded: on expiry the status word
+// gets MOE_ERR_TIMEOUT and every thread of the CTA sees false.
 // spin_limit bounds the polling (MOE_SPIN_LIMIT unless a test lowers it);
 // extra > 0 (a test setting) makes the barrier wait for arrivals that never
 // come, so that every waiter runs into that bound.
@@ -221,21 +219,17 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned ph, int sit
     __syncthreads();
     int ok = 1;
     if (threadIdx.x == 0) {
-        const unsigned G = gridDim.x, NG = min(G, (unsigned)DF_BAR_GROUPS), grp = blockIdx.x % NG;
-        const unsigned members = (G - grp + NG - 1) / NG + extra;
-        unsigned* flag = bar + 32 * (DF_BAR_GROUPS + 1);
-        __threadfence();
-        if (atomicAdd(bar + 32 * grp, 1u) + 1u == ph * members &&
-            atomicAdd(bar + 32 * DF_BAR_GROUPS, 1u) + 1u == ph * NG) {
-            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(ph) : "memory");
-        } else {
+        const unsigned target = ph * (gridDim.x + extra);
+        unsigned v;
+        // the arrival releases this CTA's writes (ordered before it by the CTA barrier);
+        // the last arrival and every waiter acquire everyone else's
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(v) : "l"(bar) : "memory");
+        if (v + 1u < target) {
             unsigned it = 0;
-            while (ld_acquire_u32(flag) < ph) {
-                if (++it > spin_limit) { moe_note_timeout(site, (int)(ld_acquire_u32(flag) % 1000)); ok = 0; break; }
-                if (it > 16) __nanosleep(32);
+            while (ld_acquire_u32(bar) < target) {
+                if (++it > spin_limit) { moe_note_timeout(site, (int)(ld_acquire_u32(bar) % 1000)); ok = 0; break; }
             }
         }
-        __threadfence();
     }
     return __syncthreads_and(ok) != 0;
 }
@@ -382,17 +376,6 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* tm, ui
             "r"(smem_u32(dst)),
         "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
         : "memory");
-}
-
-// 16 bytes global -> shared through L2 (cp.async, the LSU path).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-
-// The mbarrier's current phase also waits for this thread's earlier cp.async
-// copies (its pending count is raised now and lowered when they land).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
@@ -589,8 +572,9 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
         const int J = J0 + j;
-        uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-        if (g < T) bx = xb[(J * 4 + q) * T + g];
+        // lanes g >= T load another token's fragment (or, at the last block, the first
+        // bytes of xc, which follows xb): it only feeds MMA columns >= T, never stored
+        const uint4 bx = xb[(J * 4 + q) * T + g];
         const float4 c = xc[J * 4 + q];
         const uint32_t sel = (j & 1) ? 0x4342u : 0x4140u;  // 2-bit: the block's half of the word
         const int wi = BITS == 2 ? (j >> 1) : j;
@@ -620,8 +604,8 @@ __device__ __forceinline__ void df_compute_c(const DfCRegs<BITS>& r, const uint4
 // ---------------------------------------------------------------- phase D: one expert, one feature tile
 
 // acc (features g, g + 8; pair columns 2q, 2q + 1) = W_d rows ft .. ft + 15 x h
-// of the expert's n pairs, straight from the slot in a rolled loop (two
-// blocks per step): a W_d unit is used once per launch, so its code stays
+// of the expert's n pairs, straight from the slot in a loop of two blocks per
+// step, unrolled twice: a W_d unit is used once per launch, so its code stays
 // small instead of being unrolled over all blocks.  The unit's codes sit as
 // [16 rows][nbox 128-byte chunks] with the TMA 128-byte swizzle keyed on the
 // 128-byte line index (row * nbox + chunk); scales as [16 rows][nblk] fp16;
@@ -636,7 +620,7 @@ __device__ __forceinline__ void df_compute_d_smem(const uint8_t* code, const uin
     const bool col_ok = g < n, ok0 = 2 * q < n, ok1 = 2 * q + 1 < n;
     const int mrow = ((lane >> 3) & 1) * 8 + (lane & 7), jo = lane >> 4;  // ldmatrix row address of this lane
     const uint8_t* hrow = hs + g * hstride + q * 16;
-#pragma unroll 1
+#pragma unroll 2
     for (int j = 0; j < nblk; j += 2) {
         uint32_t c[2][2];  // [block j, j + 1][row g, g + 8]
         if (BD == 4) {
@@ -713,6 +697,7 @@ __device__ __forceinline__ DfSmem df_smem(uint8_t* smem_raw, const DfPlan& pl, i
 template <int BGU, int BD, int NBD>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     k_decode_fused(const __grid_constant__ CUtensorMap tgu, const __grid_constant__ CUtensorMap tcd,
+                   const __grid_constant__ CUtensorMap tsg, const __grid_constant__ CUtensorMap tsd,
                    DecodeFusedArgs a) {
     extern __shared__ uint8_t smem_raw[];
     constexpr int CK = df_ck(BGU), NBU = CK / 32;  // codes and quant blocks per gate/up unit
@@ -737,6 +722,10 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     const int G = gridDim.x, cta = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
+        tma_prefetch_desc(&tgu);
+        tma_prefetch_desc(&tcd);
+        tma_prefetch_desc(&tsg);
+        tma_prefetch_desc(&tsd);
         for (int i = 0; i < DF_WARPS * DF_NBUF; ++i) mbar_init(&full[i], 1);
         mbar_init(abar, 1);
         mbar_init(wbar, 1);
@@ -1084,72 +1073,89 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     const int ndw = (alive && nuq > warp) ? (nuq - warp + DF_WARPS - 1) / DF_WARPS : 0;
     const int S = nC + nftc * ndw;
     const uint32_t bytes_c = 2u * 2048u, bytes_d = (uint32_t)(nbox_d * 2048);
-    const int64_t srow_g = H / 32 * 2, srow_d = nblk_d * 2;  // bytes of a scale row (gate/up, down)
+    const uint32_t bytes_sc = 2u * 16u * NBU * 2u, bytes_sd = 16u * nblk_d * 2u;  // their scales
 
-    // Issue unit s of this warp into its slot s % DF_NBUF (all lanes): every
-    // lane copies 16 bytes of scales with cp.async, then lane 0 starts one TMA
-    // load of the codes.  The slot's barrier completes when both have landed.
-    auto issue = [&](int s) {
+    // Units of this warp in order: gate/up units ub .. ue - 1 (unit u = chunk u % NCH
+    // of local tile u / NCH; tile r0 + lt is rows r16 * 16 .. +15 of distinct expert
+    // ui), then W_d units (feature round rr, expert warp + 16 dd).  The issuing lane
+    // and the consuming warp walk them with their own cursors, without divisions.
+    struct Cur {
+        int lt, ch, ui, r16, rr, dd;
+    };
+    auto cur_init = [&](Cur& c) {
+        const int u = ub, lt = u / max(NCH, 1), gt = r0 + lt;
+        c.lt = lt;
+        c.ch = u - lt * NCH;
+        c.ui = gt / tiles_e;
+        c.r16 = gt - c.ui * tiles_e;
+        c.rr = 0;
+        c.dd = 0;
+    };
+    auto cur_next = [&](Cur& c, int s_done) {  // s_done: the unit just passed
+        if (s_done < nC) {
+            if (++c.ch == NCH) {
+                c.ch = 0;
+                ++c.lt;
+                if (++c.r16 == tiles_e) {
+                    c.r16 = 0;
+                    ++c.ui;
+                }
+            }
+        } else if (++c.dd == ndw) {
+            c.dd = 0;
+            ++c.rr;
+        }
+    };
+
+    // Issue unit s (at the issuing cursor) into this warp's slot s % DF_NBUF: one
+    // lane starts the TMA loads of its codes and its scales; the slot's barrier
+    // completes when both have landed.
+    auto issue = [&](int s, const Cur& c) {
         const int b = s % DF_NBUF;
         uint64_t* fb = &full[warp * DF_NBUF + b];
         uint8_t* cdst = ring + (warp * DF_NBUF + b) * DF_CODE_SLOT;
         uint8_t* sdst = scr + (warp * DF_NBUF + b) * pl.sc_slot;
         if (s < nC) {
-            const int u = ub + s, lt = u / NCH, ch = u % NCH, gt = r0 + lt, ui = gt / tiles_e, r16 = gt % tiles_e;
-            const int sl = rt.u_sl[ui];
-            if (sl >= 0) {
-                // scales [gate, up][16 rows][NBU]: lane l takes row l % 16 of matrix l / 16
-                const uint8_t* src = a.arena + (int64_t)sl * a.slot_bytes + a.off_scales[lane >> 4] +
-                                     (int64_t)(r16 * 16 + (lane & 15)) * srow_g + ch * NBU * 2;
-                uint8_t* dst = sdst + (lane >> 4) * 16 * NBU * 2 + (lane & 15) * NBU * 2;
-#pragma unroll
-                for (int z = 0; z < NBU / 8; ++z) cp_async16(dst + 16 * z, src + 16 * z);
-                cp_async_mbar_arrive(fb);
-            }
-            __syncwarp();
-            if (lane == 0) {
-                if (sl < 0) {
-                    mbar_arrive(fb);  // nothing to load: the unit counts 0
-                } else {
-                    mbar_arrive_expect_tx(fb, bytes_c);
-                    tma_load_5d(cdst, &tgu, fb, 0, ch, r16 * 16, 0, sl);  // gate and up, 16 rows x 128 B each
-                }
+            const int sl = rt.u_sl[c.ui];
+            if (sl < 0) {
+                mbar_arrive(fb);  // nothing to load: the unit counts 0
+            } else {
+                mbar_arrive_expect_tx(fb, bytes_c + bytes_sc);
+                tma_load_5d(cdst, &tgu, fb, 0, c.ch, c.r16 * 16, 0, sl);  // gate and up, 16 rows x 128 B each
+                tma_load_4d(sdst, &tsg, fb, c.ch * NBU, c.r16 * 16, 0, sl);  // [gate, up][16 rows][NBU] fp16
             }
         } else {
-            const int d = s - nC, rr = d / ndw, ui = warp + DF_WARPS * (d % ndw);
-            const int ft = (cta + rr * G) * DF_FT;
+            const int ui = warp + DF_WARPS * c.dd, ft = (cta + c.rr * G) * DF_FT;
             const int sl = rt.u_sl[ui];
-            if (sl >= 0) {  // scales [16 rows][nblk_d]: lane l takes 16 bytes of row l % 16
-                const int per = (int)(srow_d / 16);  // 16-byte pieces per row (1 or 2)
-                if (lane < 16 * per) {
-                    const uint8_t* src = a.arena + (int64_t)sl * a.slot_bytes + a.off_scales[2] +
-                                         (int64_t)(ft + lane % 16) * srow_d + (lane / 16) * 16;
-                    cp_async16(sdst + (lane % 16) * srow_d + (lane / 16) * 16, src);
-                }
-                cp_async_mbar_arrive(fb);
-            }
-            __syncwarp();
-            if (lane == 0) {
-                if (sl < 0) {
-                    mbar_arrive(fb);
-                } else {
-                    mbar_arrive_expect_tx(fb, bytes_d);
-                    tma_load_4d(cdst, &tcd, fb, 0, 0, ft, sl);  // 16 rows x nbox_d x 128 B
-                }
+            if (sl < 0) {
+                mbar_arrive(fb);
+            } else {
+                mbar_arrive_expect_tx(fb, bytes_d + bytes_sd);
+                tma_load_4d(cdst, &tcd, fb, 0, 0, ft, sl);  // 16 rows x nbox_d x 128 B
+                tma_load_3d(sdst, &tsd, fb, 0, ft, sl);     // [16 rows][nblk_d] fp16
             }
         }
     };
 
     int issued = 0;  // units issued by this warp (the same count in every lane)
+    Cur ic;          // the issuing lane's cursor
+    cur_init(ic);
     if (S > 0) {
-        if (lane == 0) fence_proxy_async_smem();  // the ring held generic-proxy data during A and B
-        __syncwarp();
-        for (; issued < min(S, DF_NBUF); ++issued) issue(issued);
+        if (lane == 0) {
+            fence_proxy_async_smem();  // the ring held generic-proxy data during A and B
+            for (int i = 0; i < min(S, DF_NBUF); ++i) {
+                issue(i, ic);
+                cur_next(ic, i);
+            }
+        }
+        issued = min(S, DF_NBUF);
     }
     DF_CLK(cl0);
     if (nC > 0) DF_WACC(9, cl0 - cb0);
     bool wok = true;
     int s = 0;  // units consumed
+    Cur cc;     // the consuming cursor (every lane)
+    cur_init(cc);
     {
         float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
         const int g = lane >> 2, q = lane & 3;
@@ -1161,8 +1167,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             DF_WACC(0, c1 - c0);
             DF_WACC(4, 1);
             if (s == 0) DF_MARK(10);
-            const int u = ub + s, lt = u / NCH, ch = u % NCH, gt = r0 + lt, ui = gt / tiles_e;
-            const bool valid = rt.u_sl[ui] >= 0;
+            const bool valid = rt.u_sl[cc.ui] >= 0;
             DfCRegs<BGU> cr;
             if (valid)
                 df_stage_c<BGU>(ring + (warp * DF_NBUF + b) * DF_CODE_SLOT, scr + (warp * DF_NBUF + b) * pl.sc_slot,
@@ -1170,15 +1175,21 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             __syncwarp();  // every lane's reads of the slot are done: it may be refilled
             DF_CLK(c1a);
             DF_WACC(8, c1a - c1);
-            if (issued < S) issue(issued++);  // re-arm the slot with unit s + DF_NBUF
+            if (issued < S) {  // re-arm the slot with unit s + DF_NBUF
+                if (lane == 0) {
+                    issue(issued, ic);
+                    cur_next(ic, issued);
+                }
+                ++issued;
+            }
             DF_CLK(c1b);
             DF_WACC(7, c1b - c1a);
-            if (valid) df_compute_c<BGU>(cr, xb, xc, ch * NBU, T, accg, accu);
+            if (valid) df_compute_c<BGU>(cr, xb, xc, cc.ch * NBU, T, accg, accu);
             DF_CLK(c2);
             DF_WACC(1, c2 - c1);
             if (s == 0) DF_WACC(6, c2 - c1);
-            if (s == nC - 1 || (u + 1) / NCH != lt) {  // this warp's part of tile lt is complete
-                float* pp = part + (size_t)(lt + warp) * (2 * 16 * T);  // [gate, up][16 rows][T]
+            if (s == nC - 1 || cc.ch == NCH - 1) {  // this warp's part of tile lt is complete
+                float* pp = part + (size_t)(cc.lt + warp) * (2 * 16 * T);  // [gate, up][16 rows][T]
 #pragma unroll
                 for (int z = 0; z < 2; ++z) {
                     const int col = 2 * q + z;
@@ -1193,6 +1204,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
 #pragma unroll
                 for (int z = 0; z < 4; ++z) accg[z] = accu[z] = 0.f;
             }
+            cur_next(cc, s);
         }
     }
     const bool cok = __syncthreads_and(wok && alive) != 0;
@@ -1260,7 +1272,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
             DF_CLK(c1);
             DF_WACC(2, c1 - c0);
             DF_WACC(5, 1);
-            const int d = s - nC, rr = d / ndw, ui = warp + DF_WARPS * (d % ndw);
+            const int rr = cc.rr, ui = warp + DF_WARPS * cc.dd;
             const int pos0 = rt.u_pos[ui], n = rt.u_n[ui];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             if (rt.u_sl[ui] >= 0)
@@ -1268,7 +1280,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                                            scr + (warp * DF_NBUF + b) * pl.sc_slot, hs + (size_t)pos0 * pl.hs_stride,
                                            pl.hs_stride, hsum + (size_t)pos0 * nblk_d, n, acc);
             __syncwarp();  // the slot's reads are done: it may be refilled
-            if (issued < S) issue(issued++);
+            if (issued < S) {
+                if (lane == 0) {
+                    issue(issued, ic);
+                    cur_next(ic, issued);
+                }
+                ++issued;
+            }
             DF_CLK(c2);
             DF_WACC(3, c2 - c1);
 #pragma unroll
@@ -1282,6 +1300,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                     yp[g + 8] = wv * acc[2 + z];
                 }
             }
+            cur_next(cc, s);
         }
         alive = __syncthreads_and(wok) != 0;
         DF_MARK(15);

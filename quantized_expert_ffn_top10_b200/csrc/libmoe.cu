@@ -245,6 +245,33 @@ bool tmap_codes_d(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Gate and up scales of every slot as one 4-D fp16 tensor (block, row, matrix,
+// slot); a box is nblk blocks of 16 rows of both matrices, landing as
+// [matrix][row][nblk].
+bool tmap_scales_gu(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t nblk_row, int64_t mat_stride,
+                    int64_t n_slots, int64_t slot_bytes, int nblk) {
+    cuuint64_t dims[4] = {(cuuint64_t)nblk_row, (cuuint64_t)rows, 2, (cuuint64_t)n_slots};
+    cuuint64_t strides[3] = {(cuuint64_t)nblk_row * 2, (cuuint64_t)mat_stride, (cuuint64_t)slot_bytes};
+    cuuint32_t box[4] = {(cuuint32_t)nblk, 16, 2, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// W_d scales of every slot as a 3-D fp16 tensor (block, row, slot); a box is
+// the whole scale row of 16 rows, landing as [row][nblk].
+bool tmap_scales_d(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t nblk_row, int64_t n_slots,
+                   int64_t slot_bytes) {
+    cuuint64_t dims[3] = {(cuuint64_t)nblk_row, (cuuint64_t)rows, (cuuint64_t)n_slots};
+    cuuint64_t strides[2] = {(cuuint64_t)nblk_row * 2, (cuuint64_t)slot_bytes};
+    cuuint32_t box[3] = {(cuuint32_t)nblk_row, 16, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -363,6 +390,9 @@ bool fused_decode_ok(const moe_arena_desc* d, int T, int E, int k, DfPlan* plan,
     const int H = d->H, I = d->I, G = g_df_grid[dev];
     if (d->bits_gate != d->bits_up) return false;  // one unit shape for gate and up
     if (d->off_codes[1] <= d->off_codes[0]) return false;  // gate and up codes as one tensor
+    if (d->off_scales[1] <= d->off_scales[0] || (d->off_scales[1] - d->off_scales[0]) % 16 ||
+        d->off_scales[0] % 16 || d->off_scales[2] % 16)
+        return false;  // gate and up scales as one tensor; every scale tensor 16-byte aligned
     if (T > DF_TN || T * k > DF_MAXP || E > MOE_MAX_E || H > kDfMaxH) return false;
     if (H % df_ck(d->bits_gate) || H % 256 || I % 256 || I / 32 > DF_MAX_NBD) return false;
     const int wd_row = I * d->bits_down / 8;  // bytes of a W_d row: one or two 128-byte boxes
@@ -385,7 +415,7 @@ cudaError_t launch_fused(const CUtensorMap* tm, const DecodeFusedArgs& a, int gr
     at[0].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_fused<BGU, BD, NBD>, tm[0], tm[1], a);
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<BGU, BD, NBD>, tm[0], tm[1], tm[2], tm[3], a);
 }
 
 int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
@@ -417,11 +447,14 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     a.pl = plan;
     a.spin_limit = g_dbg_spin.load() ? g_dbg_spin.load() : MOE_SPIN_LIMIT;
     a.bar1_extra = g_dbg_bar1.load();
-    CUtensorMap tm[2];
+    CUtensorMap tm[4];
     const int64_t ns = d->n_slots, sb = d->slot_bytes;
     if (!tmap_codes_gu(&tm[0], c.arena + d->off_codes[0], I, (int64_t)H * d->bits_gate / 8,
                        d->off_codes[1] - d->off_codes[0], ns, sb) ||
-        !tmap_codes_d(&tm[1], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb))
+        !tmap_codes_d(&tm[1], c.arena + d->off_codes[2], H, (int64_t)I * d->bits_down / 8, ns, sb) ||
+        !tmap_scales_gu(&tm[2], c.arena + d->off_scales[0], I, H / 32, d->off_scales[1] - d->off_scales[0], ns, sb,
+                        df_ck(d->bits_gate) / 32) ||
+        !tmap_scales_d(&tm[3], c.arena + d->off_scales[2], H, I / 32, ns, sb))
         return MOE_ERR_CUDA;
     // the grid barrier's words and the recheck counter start at zero: one memset when the
     // counter is the workspace's own (it sits just before the barrier words), else two

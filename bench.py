@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-decode", action="store_true", help="profiling runs: no decode sections")
     p.add_argument("--no-stacks", action="store_true", help="skip the two 48-layer stacks")
+    p.add_argument("--no-midt", action="store_true", help="skip the mid-T (T = 16, 64, 256) prefill lines")
     p.add_argument("--no-cpu-baseline", action="store_true", help="profiling runs: skip the oracle timing")
     p.add_argument("--decode-layers", type=int, default=DECODE_LAYERS,
                    help="rotating decode layer arenas (profiling runs use 1)")
@@ -462,6 +463,8 @@ def run_ours(args):
         line["decode_T1"] = decode_t1_section(args, rank, local, world, dist, pk, K, W, base)
     if not args.no_prefill:
         prefill_section(args, line, rank, local, world, dist, pk, K, W, base)
+        if not args.no_midt:
+            line["prefill_midT"] = midt_section(args, rank, local, world, dist, pk, K, W)
     if not args.no_stacks:
         if not args.no_decode:
             line["decode_stack"] = decode_stack_section(args, rank, local, world, dist, pk, W, base)
@@ -592,6 +595,40 @@ def prefill_section(args, line, rank, local, world, dist, pk, K, W, base):
         line["prefill"]["cpu_baseline"] = cpu_baseline(pl, 0, 16, "16 tokens of the 8,192-token chunk, full layer")
     del pl
     torch.cuda.empty_cache()
+
+
+MIDT = (16, 64, 256)
+
+
+def midt_section(args, rank, local, world, dist, pk, K, W):
+    """Mid-T chunks (batched verify windows, short prompts) through the prefill
+    entry point at the model's shape.  With 1-14 pairs per expert the layer
+    reads each selected expert's weights once for a handful of columns, so the
+    roofline is HBM: bytes = the distinct selected experts' slots + the router
+    + x in and out, over the layer call's device time."""
+    import torch
+    import moe_synth as S
+    hbm, _, _, src = pk
+    NLd = max(1, args.decode_layers)
+    sec = {"workload": "prefill entry point, 1 layer, E=512, top_k=10, H=2048, I=512, 4-bit, Gaussian router; "
+                       f"{NLd} rotating layer arenas with fresh inputs", "graph": "one CUDA graph per layer call"}
+    for T in MIDT:
+        dl = Layers(S.config("prefill", T=T), NLd, rank)
+        c = dl.cfg
+        ms, stages, distinct, per_call, clk = time_graphs(dl, K, W, local, dist)
+        nbytes = statistics.mean(decode_bytes(c, d) for d in distinct)
+        step_ms = ms / K
+        sec[f"T{T}"] = {
+            "value": round(whole_job_rate(c.T * K, world, ms), 1), "unit": "tokens/s", "steps": K,
+            "ms_per_step": round(step_ms, 5), "distinct_experts": statistics.mean(distinct),
+            "roofline": {"bound": "hbm", "achieved": round(nbytes / (step_ms * 1e6), 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(nbytes / (step_ms * 1e6) / hbm, 4), "peak_source": src,
+                         "bytes": int(nbytes)},
+            "stage_ms": [round(statistics.mean(s[j] for s in stages), 5) for j in range(4)],
+            "gpu_launches": per_call * K, "clocks": clk}
+        del dl
+        torch.cuda.empty_cache()
+    return sec
 
 
 def decode_stack_section(args, rank, local, world, dist, pk, W, base):

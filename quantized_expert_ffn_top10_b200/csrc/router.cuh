@@ -227,8 +227,21 @@ __device__ __forceinline__ double logit_fp64_exact(const TopkArgs& a, int t, int
     const uint16_t* xr = a.x + (size_t)t * a.H;
     const float* wr = a.W + (size_t)e * a.H;
     double s = 0.0;
-#pragma unroll 8
-    for (int h = 0; h < a.H; ++h) s = fma((double)bf16_bits_to_f32(xr[h]), (double)__ldg(wr + h), s);
+    // in order over h; 8 elements per step by vector loads (H % 8 == 0, rows 16-byte aligned)
+#pragma unroll 4
+    for (int h = 0; h < a.H; h += 8) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + h));
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr + h));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr + h + 4));
+        s = fma((double)__uint_as_float(xv.x << 16), (double)w0.x, s);
+        s = fma((double)__uint_as_float(xv.x & 0xffff0000u), (double)w0.y, s);
+        s = fma((double)__uint_as_float(xv.y << 16), (double)w0.z, s);
+        s = fma((double)__uint_as_float(xv.y & 0xffff0000u), (double)w0.w, s);
+        s = fma((double)__uint_as_float(xv.z << 16), (double)w1.x, s);
+        s = fma((double)__uint_as_float(xv.z & 0xffff0000u), (double)w1.y, s);
+        s = fma((double)__uint_as_float(xv.w << 16), (double)w1.z, s);
+        s = fma((double)__uint_as_float(xv.w & 0xffff0000u), (double)w1.w, s);
+    }
     if (a.b) s += (double)a.b[e];
     return s;
 }
@@ -510,15 +523,24 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = ab[j] = 0.0;
             const uint16_t* xr = a.x + (size_t)t * H;
-#pragma unroll 4
-            for (int h = lane; h < H; h += 32) {
-                const double xd = bf16_bits_to_f32(xr[h]);
+            // lane l takes h = 4 l + 128 i .. + 3 (H % 4 == 0, rows 16-byte aligned): one
+            // 8-byte x load and one 16-byte row load per candidate keep all of a step's
+            // loads in flight; each lane still adds H / 32 products
+            for (int h0 = 4 * lane; h0 < H; h0 += 128) {
+                const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + h0));
+                const double x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+                const double x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+                float4 wv[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (base + j < NR) wv[j] = __ldg(reinterpret_cast<const float4*>(a.W + (size_t)ej[j] * H + h0));
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     if (base + j < NR) {
-                        const double p = xd * (double)__ldg(a.W + (size_t)ej[j] * H + h);
-                        acc[j] += p;
-                        ab[j] += fabs(p);
+                        const double p0 = x0 * (double)wv[j].x, p1 = x1 * (double)wv[j].y;
+                        const double p2 = x2 * (double)wv[j].z, p3 = x3 * (double)wv[j].w;
+                        acc[j] += p0; acc[j] += p1; acc[j] += p2; acc[j] += p3;
+                        ab[j] += fabs(p0); ab[j] += fabs(p1); ab[j] += fabs(p2); ab[j] += fabs(p3);
                     }
             }
 #pragma unroll

@@ -69,7 +69,7 @@ def _sample_tokens(T, idx, E, rng, n=48):
     return np.array(sorted(pick), np.int32)
 
 
-def _full_size(cfg, layer=0):
+def _full_size(cfg, layer=0, all_tokens=False):
     import torch
     wl = Workload(cfg)
     x = wl.x_host()
@@ -82,7 +82,10 @@ def _full_size(cfg, layer=0):
     ref_hist = np.zeros((cfg.L, cfg.E), np.uint32)
     O.hist_add(counts, layer, ref_hist)
     assert np.array_equal(hist.cpu().numpy().view(np.uint32), ref_hist)
-    toks = _sample_tokens(cfg.T, idx, cfg.E, np.random.default_rng(cfg.seed))
+    if all_tokens:
+        toks = np.arange(cfg.T, dtype=np.int32)
+    else:
+        toks = _sample_tokens(cfg.T, idx, cfg.E, np.random.default_rng(cfg.seed), n=min(48, cfg.T))
     ref = wl.oracle_layer(layer, x, tokens=toks)
     assert np.array_equal(ref["idx"][toks], idx[toks])
     assert_out_close(out, ref["out_f64"], rows=toks)
@@ -93,6 +96,21 @@ def test_prefill_full_chunk_uniform(cuda_ok):
     """8,192 tokens, E = 512, 4-bit, Gaussian router (about 160 tokens per expert)."""
     counts = _full_size(S.config("prefill"))
     assert counts.sum() == 8192 * 10
+
+
+@pytest.mark.parametrize("T", [16, 64, 256])
+def test_prefill_mid_T_model_shape(cuda_ok, T):
+    """Mid-T chunks (batched verify windows, short prompts) at the model's shape:
+    E = 512, H = 2048, I = 512, 4-bit, Gaussian router.  With 160 to 2,560 pairs
+    over 512 experts most experts get 0 to 5 pairs, so nearly every grouped-GEMM
+    tile is a single ragged column block.  Routing of every token bit-exact, the
+    histogram bit-exact, and the outputs of every token (T <= 64) or of 48
+    sampled tokens plus every token of the two most and two least loaded experts."""
+    counts = _full_size(S.config("prefill", T=T, seed=70 + T), all_tokens=T <= 64)
+    assert counts.sum() == T * 10
+    used = counts[counts > 0]
+    assert used.max() <= 40 and used.min() >= 1
+    assert (counts > 0).sum() >= min(T * 10 // 2, 300)
 
 
 def _pair_outputs(ws, cfg, T, sel):

@@ -24,7 +24,7 @@ inline size_t al(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
     size_t idx, w, logit, absum, cmax, offsets, perm, inv, uniq, meta, chunk, tiles, nrechk, xp, h, y, rec, gbar, wsplit,
-        xn, slow, hout, reck, total;
+        xn, slow, slowrec, last, hout, reck, total;
 };
 
 inline int max_tiles(int P, int E) { return (P + PREFILL_TILE_N - 1) / PREFILL_TILE_N + std::min(E, P); }
@@ -58,6 +58,8 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     w.wsplit = put(small ? 0 : (size_t)3 * E * H * 2);        // chunk router: W_r as three bf16 planes
     w.xn = put(small ? 0 : (size_t)T * 4);                     // chunk router: ||x_t|| per token
     w.slow = put(small ? 0 : (size_t)(T + 4) * 4);             // chunk top-k: [count, tokens...] left to the slow pass
+    w.slowrec = put(small ? 0 : (size_t)T * sizeof(SlowRec));  // and the fast pass's candidates of each
+    w.last = put(small ? 0 : (size_t)(T + 4) * 4);             // [count, tokens...] left to the last pass
     w.hout = put(small ? (size_t)T * H * 4 : 0);               // fused decode + steering: fp32 output rows
     w.total = o;
     return w;
@@ -170,9 +172,15 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
         ta.xnorm = xn;
         ta.slow_count = reinterpret_cast<int32_t*>(ws + L.slow);
         ta.slow_list = ta.slow_count + 4;
-        if (cudaMemsetAsync(ta.slow_count, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+        ta.slow_rec = reinterpret_cast<SlowRec*>(ws + L.slowrec);
+        ta.last_count = reinterpret_cast<int32_t*>(ws + L.last);
+        ta.last_list = ta.last_count + 4;
+        if (cudaMemsetAsync(ta.slow_count, 0, 4, st) != cudaSuccess ||
+            cudaMemsetAsync(ta.last_count, 0, 4, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
         k_topk_fast<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
-        k_topk_slow<0><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+        k_topk_slow<<<std::min(T, 4 * 148), 32 * MOE_SLOW_WARPS, 0, st>>>(ta);
+        k_topk_last<<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     }
     PermArgs pa{};
     pa.idx = idx; pa.P = P; pa.E = E; pa.nchunks = (P + PERM_CHUNK - 1) / PERM_CHUNK;
@@ -186,7 +194,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
     k_perm_count<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
     k_perm_scan<<<1, MOE_MAX_E, 0, st>>>(pa);
     k_perm_scatter<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
-    count(T <= MOE_DECODE_MAX_T ? 5 : 8);
+    count(T <= MOE_DECODE_MAX_T ? 5 : 9);
     return cuda_rc(cudaGetLastError());
 }
 

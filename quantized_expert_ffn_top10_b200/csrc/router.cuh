@@ -13,6 +13,8 @@
 // fused multiply-add sequence reproduces it bit for bit), and the selection is
 // taken on those values with ties going to the lower expert index.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 #define MOE_TOPK_WARPS 4
@@ -173,6 +175,18 @@ __global__ void __launch_bounds__(256) k_router_gemm(const uint16_t* __restrict_
 
 // ---------------------------------------------------------------- certified top-k
 
+// What the fast pass knows about a token it could not certify: its M
+// candidates in rank order (value desc, expert asc) and an upper end of
+// everything else, so that the slow pass starts at the re-evaluation.
+struct SlowRec {
+    double val[32];  // fast values
+    double bnd[32];  // their error bounds
+    int32_t e[32];   // experts
+    double rest;     // upper end of every non-candidate (-inf when none)
+    int32_t mc;      // number of candidates
+    int32_t pad;
+};
+
 struct TopkArgs {
     const uint16_t* x;      // [T][H] bf16
     const float* W;         // [E][H]
@@ -186,6 +200,9 @@ struct TopkArgs {
     int32_t* n_rechecked;   // [1]
     int32_t* slow_list;     // tokens the fast pass could not certify (k_topk_fast), or null
     int32_t* slow_count;    // [1] their number (zeroed before the fast pass)
+    SlowRec* slow_rec;      // [T] the fast pass's candidates of each listed token
+    int32_t* last_list;     // tokens the slow pass could not certify either (k_topk_last)
+    int32_t* last_count;    // [1] their number (zeroed before the fast pass)
     double gfast;           // gamma_n of the fast logits' summation
     int T, H, E, k;
 };
@@ -305,6 +322,46 @@ __device__ __forceinline__ bool sort_and_certify(double& cval, double& cbnd, int
     return certify_sorted(cval, cbnd, M, k, rest);
 }
 
+// Lanes hold M candidates in rank order after a failed certification.  The
+// candidates to re-evaluate exactly: both ends of every overlapping adjacent
+// pair among the k + 1 best, and candidates further down whose interval
+// reaches the k-th (which then needs its own value too).  Returns the lane mask.
+__device__ __forceinline__ unsigned reeval_mask(double cval, double cbnd, int MC, int k) {
+    const int lane = threadIdx.x & 31;
+    const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
+    const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
+    const double lok = __shfl_sync(0xffffffffu, lo_end(cval, cbnd), k - 1);
+    const bool pairbad = lane < k && lane + 1 < MC && !(lo_end(cval, cbnd) > hi_end(nv, nb));
+    const bool tailbad = lane > k && lane < MC && !(lok > hi_end(cval, cbnd));
+    const bool anytail = __any_sync(0xffffffffu, tailbad);
+    const bool prevup = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0;
+    const bool prevbad = (prevup && lane > 0) || (lane == k - 1 && anytail);
+    return __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad || tailbad));
+}
+
+// One warp: x_t . W[e] in fp64, lanes taking h = 4 l + 128 i .. + 3 (each lane
+// adds H / 32 products), and the sum of the products' magnitudes, both
+// reduced over the warp (every lane gets them).
+__device__ __forceinline__ void dot_fp64_warp(const TopkArgs& a, int t, int e, double& s, double& sa) {
+    const int lane = threadIdx.x & 31, H = a.H;
+    const uint16_t* xr = a.x + (size_t)t * H;
+    const float* wr = a.W + (size_t)e * H;
+    double acc = 0.0, ab = 0.0;
+#pragma unroll 4
+    for (int h0 = 4 * lane; h0 < H; h0 += 128) {
+        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + h0));
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(wr + h0));
+        const double p0 = (double)__uint_as_float(xv.x << 16) * (double)wv.x;
+        const double p1 = (double)__uint_as_float(xv.x & 0xffff0000u) * (double)wv.y;
+        const double p2 = (double)__uint_as_float(xv.y << 16) * (double)wv.z;
+        const double p3 = (double)__uint_as_float(xv.y & 0xffff0000u) * (double)wv.w;
+        acc += p0; acc += p1; acc += p2; acc += p3;
+        ab += fabs(p0); ab += fabs(p1); ab += fabs(p2); ab += fabs(p3);
+    }
+    s = warp_sum_d(acc);
+    sa = warp_sum_d(ab);
+}
+
 __device__ __forceinline__ void write_topk(int k, double cval, int ce, int32_t* idx_out, float* w_out) {
     const int lane = threadIdx.x & 31;
     const double v0 = __shfl_sync(0xffffffffu, cval, 0);
@@ -359,7 +416,10 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             xnorm = sqrtf(s) * 1.001f;
         }
     }
-    double v[NV], dl[NV];
+    // fp32 fast logits (MODE 0) are held in fp32 with their bounds rounded up to
+    // fp32: half the registers of fp64 values, and the intervals only widen
+    using VT = typename std::conditional<F64, double, float>::type;
+    VT v[NV], dl[NV];
     uint32_t key[NV];  // order-preserving 32-bit keys of the values rounded to fp32
     uint32_t taken = 0;
 #pragma unroll
@@ -374,11 +434,12 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
             } else {
                 f = static_cast<const float*>(a.logit)[(size_t)t * E + e];
                 if (isnan(f)) f = -INFINITY;
-                v[i] = (double)f;
+                v[i] = f;
             }
             if (MODE == 1) B = a.absum[(size_t)t * E + e] * (1.0 + 1e-9);
             else B = ((double)xnorm * (double)a.wnorm[e] + (a.b ? fabs((double)a.b[e]) : 0.0)) * 1.001;
-            dl[i] = order_bnd(B * (a.gfast + g_or) + 1e-300);
+            const double bd = order_bnd(B * (a.gfast + g_or) + 1e-300);
+            dl[i] = F64 ? (VT)bd : (VT)__double2float_ru(bd);
             const uint32_t u = __float_as_uint(f);
             key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         } else {
@@ -488,7 +549,20 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
         return;
     }
     if (FAST_ONLY) {
-        if (lane == 0) a.slow_list[atomicAdd(a.slow_count, 1)] = t;
+        int slot = 0;
+        if (lane == 0) {
+            slot = atomicAdd(a.slow_count, 1);
+            a.slow_list[slot] = t;
+        }
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        SlowRec* r = a.slow_rec + slot;
+        r->val[lane] = cval;
+        r->bnd[lane] = cbnd;
+        r->e[lane] = ce;
+        if (lane == 0) {
+            r->rest = rest;
+            r->mc = MC;
+        }
         return;
     }
     // 3) prefill: re-evaluate in fp64 (lane-strided) the candidates that the
@@ -498,17 +572,7 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int t, int32_t* id
     //    which still contain the exact logits, so the second certification
     //    below is as valid as the first.
     if (MODE == 0) {
-        const double nv = __shfl_down_sync(0xffffffffu, cval, 1);
-        const double nb = __shfl_down_sync(0xffffffffu, cbnd, 1);
-        const double lok = __shfl_sync(0xffffffffu, lo_end(cval, cbnd), k - 1);
-        // overlapping adjacent pairs among the k + 1 best, and candidates further
-        // down whose interval reaches the k-th (which then needs its own value too)
-        const bool pairbad = lane < k && lane + 1 < MC && !(lo_end(cval, cbnd) > hi_end(nv, nb));
-        const bool tailbad = lane > k && lane < MC && !(lok > hi_end(cval, cbnd));
-        const bool anytail = __any_sync(0xffffffffu, tailbad);
-        const bool prevup = __shfl_up_sync(0xffffffffu, pairbad ? 1 : 0, 1) != 0;
-        const bool prevbad = (prevup && lane > 0) || (lane == k - 1 && anytail);
-        const unsigned need = __ballot_sync(0xffffffffu, lane < MC && (pairbad || prevbad || tailbad));
+        const unsigned need = reeval_mask(cval, cbnd, MC, k);
         const int NR = __popc(need);
         for (int base = 0; base < NR; base += 16) {
             int ej[16], lj[16];
@@ -642,16 +706,78 @@ __global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk_fast(TopkArgs a) {
     topk_token<MODE, true>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
 }
 
-// The tokens k_topk_fast listed, one warp each (launched for up to T of them).
-template <int MODE>
-__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk_slow(TopkArgs a) {
+// The tokens k_topk_fast listed (prefill fast logits), one CTA each, looping
+// over the list: warp 0 takes the fast pass's ranked candidates and flags the
+// ones to re-evaluate, every warp re-evaluates some of them in fp64, and warp 0
+// certifies again; a token that still does not certify goes to k_topk_last.
+#define MOE_SLOW_WARPS 8
+__global__ void __launch_bounds__(32 * MOE_SLOW_WARPS) k_topk_slow(TopkArgs a) {
+    __shared__ int s_list[32];
+    __shared__ int s_e[32];
+    __shared__ double s_v[32], s_b[32];
+    __shared__ int s_nr;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const double u64 = 1.1102230246251565e-16;
+    const double g_or = (double)(a.H + 2) * u64 * 1.01;         // the definition's own rounding
+    const double g_par = (double)(a.H / 32 + 8) * u64 * 1.01;   // warp-parallel fp64 sums
+    const int n = *a.slow_count;
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const int t = a.slow_list[i];
+        const SlowRec* r = a.slow_rec + i;
+        double cval = -INFINITY, cbnd = 0.0;
+        int ce = 0x7fffffff, MC = 0;
+        double rest = 0.0;
+        if (warp == 0) {
+            MC = r->mc;
+            rest = r->rest;
+            if (lane < MC) {
+                cval = r->val[lane];
+                cbnd = r->bnd[lane];
+                ce = r->e[lane];
+            }
+            const unsigned need = reeval_mask(cval, cbnd, MC, a.k);
+            if ((need >> lane) & 1u) s_list[__popc(need & ((1u << lane) - 1))] = lane;
+            s_e[lane] = ce;
+            if (lane == 0) s_nr = __popc(need);
+        }
+        __syncthreads();
+        const int NR = s_nr;
+        for (int q = warp; q < NR; q += MOE_SLOW_WARPS) {
+            const int j = s_list[q], e = s_e[j];
+            double sm, sa;
+            dot_fp64_warp(a, t, e, sm, sa);
+            if (lane == 0) {
+                const double bb = a.b ? (double)a.b[e] : 0.0;
+                s_v[j] = order_val(sm + bb);
+                s_b[j] = order_bnd((sa + fabs(bb)) * (1.0 + 1e-9) * (g_par + g_or) + 1e-300);
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            for (int q = 0; q < NR; ++q)
+                if (s_list[q] == lane) {
+                    cval = s_v[lane];
+                    cbnd = s_b[lane];
+                }
+            if (sort_and_certify(cval, cbnd, ce, MC, a.k, rest))
+                write_topk(a.k, cval, ce, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k);
+            else if (lane == 0)
+                a.last_list[atomicAdd(a.last_count, 1)] = t;
+        }
+        __syncthreads();  // the shared lists are reused by the next token
+    }
+}
+
+// The tokens k_topk_slow could not certify, one warp each: the whole
+// single-warp path of topk_token, its exact fallback included.
+__global__ void __launch_bounds__(32 * MOE_TOPK_WARPS) k_topk_last(TopkArgs a) {
     __shared__ int s_ce[MOE_TOPK_WARPS][MOE_MAX_E];
     __shared__ double s_cv[MOE_TOPK_WARPS][MOE_MAX_E];
     const int wid = threadIdx.x >> 5;
     const int i = blockIdx.x * MOE_TOPK_WARPS + wid;
-    if (i >= *a.slow_count) return;
-    const int t = a.slow_list[i];
-    topk_token<MODE>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
+    if (i >= *a.last_count) return;
+    const int t = a.last_list[i];
+    topk_token<0>(a, t, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k, s_ce[wid], s_cv[wid], a.n_rechecked);
 }
 
 // One warp per token.

@@ -477,9 +477,10 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-DECODE_DTYPE = ("u4/u2 codes; decode: bf16 x bf16 mma.sync on exact (128 + code) and x, fp32 accumulation, "
-                "scales applied in fp32, h rounded to bf16; prefill: bf16 tcgen05 MMA on dequantised weights, "
-                "fp32 accumulation in TMEM, h and per-pair outputs in bf16; output bf16")
+DECODE_DTYPE = ("u4/u2 codes; decode: gate/up fp16 x fp16 mma.sync on exact (1024 + code) and power-of-two "
+                "scaled x, down bf16 x bf16 mma.sync on exact (128 + code) and h, fp32 accumulation, scales "
+                "applied in fp32, h rounded to bf16; router fp64 (tensor-core DMMA); prefill: bf16 tcgen05 MMA "
+                "on dequantised weights, fp32 accumulation in TMEM, h and per-pair outputs in bf16; output bf16")
 
 
 def decode_section(args, rank, local, world, dist, pk, K, W, base):

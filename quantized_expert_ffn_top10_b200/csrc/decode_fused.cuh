@@ -12,12 +12,13 @@
 //   C  gate/up + SwiGLU: each CTA owns a contiguous range of 16-row tiles of
 //      the selected experts, cut into units of 16 rows x one 128-byte code
 //      box per matrix.  Every warp owns a contiguous run of those units and
-//      streams them itself through two private TMA slots: it waits for a
-//      unit, copies it into registers, re-arms the slot with its next unit
-//      and only then computes, so both slots of every warp are in flight
-//      almost all the time.  Partial tile sums go to shared memory and are
-//      finished (SwiGLU, bf16 h) once the CTA's warps are done.  A warp that
-//      runs out of C units already loads its first W_d units.
+//      streams them itself through two private TMA slots (codes and scales,
+//      issued by one lane): it waits for a unit, copies it into registers,
+//      re-arms the slot with its next unit and only then computes, so both
+//      slots of every warp are in flight almost all the time.  Partial tile
+//      sums go to shared memory and are finished (SwiGLU, bf16 h) once the
+//      CTA's warps are done.  A warp that runs out of C units already loads
+//      its first W_d units.
 //   -- barrier --
 //   D  down + combine: each CTA owns 16 output features (a feature tile) for
 //      every selected expert, so it holds complete sums and writes out[t][f]
@@ -25,12 +26,13 @@
 //      shared memory from L2; warps take experts round-robin with the same
 //      two-slot streaming.
 //
-// The dot products run on mma.sync m16n8k16 (bf16 in, fp32 out) with the
-// weights as A (16 rows) and the tokens (or an expert's pairs) as the 8
-// columns of B, so a weight costs its unpack and one lane-slot of an MMA.
-// Codes enter the MMA as (128 + q) in bf16 (an exponent-bias bit pattern:
-// 0x4300 | q), so each block's MMA result is sum q x + 128 sum x; the block
-// correction (128 + offset) * sum x enters as the MMA's C input and the
+// The dot products run on mma.sync m16n8k16 (fp32 out) with the weights as A
+// (16 rows) and the tokens (or an expert's pairs) as the 8 columns of B, so a
+// weight costs its unpack and one lane-slot of an MMA.  Gate/up codes enter
+// as fp16 (1024 + m q) (bit pattern 0x6400 | field, m = 1 or 16 by the
+// code's bit position, see unpack8_f16) against x' / m, x' a per-token
+// power-of-two multiple of x; W_d codes enter as bf16 (128 + q) (0x4300 | q)
+// against h.  Each block's offset term enters as the MMA's C input and the
 // block scale is applied in fp32.  All waits (mbarriers, grid barriers) are
 // bounded.
 #pragma once

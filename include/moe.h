@@ -52,6 +52,10 @@ extern "C" {
 #define MOE_ERR_TIMEOUT (-7)  /* a bounded device-side wait expired             */
 #define MOE_ERR_STATIC (-8)   /* size beyond moe_route_static's fixed scratch    */
 
+#define MOE_SLOT_REMOTE (-2)  /* slot-table entry: the expert lives on another GPU
+                                 (expert parallelism): it contributes zero to this
+                                 GPU's partial sums and is not an error            */
+
 #define MOE_MAX_E 512         /* experts per layer                              */
 #define MOE_MAX_TOPK 32
 #define MOE_DECODE_MAX_T 8    /* decode path: a verify window of 1 + 4 drafts fits */
@@ -200,6 +204,39 @@ int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int
  * write: calls (and forward calls with hist != NULL) that add to the same
  * hist must be ordered, e.g. on one stream; concurrent ones lose counts.
  */
+/*
+ * Expert parallelism: experts e mod G on G GPUs, the router replicated, an
+ * all-gather of x and a reduce-scatter of fp32 partial outputs (the "Picking
+ * a quant" page's multi-GPU section gives splitting a model over GPUs as
+ * prior art; the layer's arithmetic is moe_forward_decode's).  Each GPU calls moe_forward_partial on the
+ * gathered tokens with a slot table in which the experts it does not hold are
+ * MOE_SLOT_REMOTE; the caller sums the G partials (a reduce-scatter) and
+ * moe_finish_rows adds the residual and rounds.
+ *
+ * moe_forward_partial: the same arguments as moe_forward_decode (prefill != 0:
+ * as moe_forward_prefill) except that there is no residual, no steering and
+ * no bf16 output: partial [T][H] fp32 (device, 16-B aligned) receives, per
+ * token, the gate-weighted sum of its selected experts' outputs over the
+ * experts whose slot is held here, in slot order (the combine of the
+ * forwards before its residual and its rounding).  The routing (and
+ * route_out, hist) covers all k selections of every token, remote ones
+ * included, so every GPU sees the same routing.  Errors as the forwards.
+ */
+int moe_forward_partial(int prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table,
+                        int L, int layer, const uint16_t* x, int T, const float* router_w,
+                        const float* router_bias, int E, int top_k, float* partial, uint32_t* hist,
+                        const moe_route_out* route_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * out[t][c] = bf16((residual ? x[t][c] : 0) + sum[t][c]) for T rows of H,
+ * with the steering projection applied first when steer != NULL (as in the
+ * forwards: r - (r . v) v on the fp32 row, residual included).  x [T][H] bf16,
+ * sum [T][H] fp32, steer [H] fp32 or NULL, out [T][H] bf16, all device,
+ * 16-B aligned; H % 8 == 0.  The finishing step of an expert-parallel layer.
+ */
+int moe_finish_rows(const uint16_t* x, const float* sum, int T, int H, int residual, const float* steer,
+                    uint16_t* out, void* stream);
+
 int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, uint32_t* hist,
                         void* stream);
 

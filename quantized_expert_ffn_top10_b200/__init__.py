@@ -46,7 +46,9 @@ EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forwar
            "moe_route_histogram", "moe_rank_experts", "moe_last_device_error", "moe_strerror",
            "moe_set_stage_events", "moe_launch_count", "moe_timeout_site", "moe_route_static",
            "moe_debug_set", "moe_workspace_offset", "moe_router_gamma", "moe_profile_bytes",
-           "moe_profile_write", "moe_profile_read", "moe_profile_hit_rate")
+           "moe_profile_write", "moe_profile_read", "moe_profile_hit_rate", "moe_forward_partial",
+           "moe_finish_rows")
+MOE_SLOT_REMOTE = -2
 MOE_DBG_SPIN_LIMIT, MOE_DBG_BARRIER_EXTRA = 1, 2
 MOE_WS_FAST_LOGITS, MOE_WS_PAIR_OUT, MOE_WS_SLOW_COUNT = 1, 2, 3
 
@@ -82,6 +84,11 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_decode.argtypes = fwd
         L.moe_forward_prefill.restype = i32
         L.moe_forward_prefill.argtypes = fwd
+        L.moe_forward_partial.restype = i32
+        L.moe_forward_partial.argtypes = [i32, P, P, P, i32, i32, P, i32, P, P, i32, i32, P, P, P, P,
+                                          ctypes.c_size_t, P]
+        L.moe_finish_rows.restype = i32
+        L.moe_finish_rows.argtypes = [P, P, i32, i32, i32, P, P, P]
         L.moe_route_histogram.restype = i32
         L.moe_route_histogram.argtypes = [P, i32, i32, i32, P, P]
         L.moe_rank_experts.restype = i32
@@ -200,6 +207,30 @@ def moe_forward_prefill(desc: ArenaDesc, arena, slot_table, L, layer, x, router_
     return _forward(lib().moe_forward_prefill, "moe_forward_prefill", desc, arena, slot_table, L, layer, x,
                     router_w, router_bias, top_k, residual, out, hist, route_out, ws, stream, raise_on_error,
                     steer=steer)
+
+
+def moe_forward_partial(prefill, desc: ArenaDesc, arena, slot_table, L, layer, x, router_w, router_bias, top_k,
+                        partial, hist=None, route_out=None, ws=None, stream=None, raise_on_error=True):
+    """Expert parallelism: partial [T, H] fp32 receives each token's gate-weighted
+    sum over the experts held here (slot != MOE_SLOT_REMOTE), no residual."""
+    T, E = x.shape[0], router_w.shape[0]
+    ro = None
+    if route_out is not None:
+        ro = RouteOut(*[_ptr(route_out.get(k)) for k in ("topk_idx", "topk_w", "expert_offsets", "perm",
+                                                          "n_rechecked")])
+    rc = lib().moe_forward_partial(int(bool(prefill)), ctypes.byref(as_desc(desc)), _ptr(arena), _ptr(slot_table),
+                                   L, layer, _ptr(x), T, _ptr(router_w), _ptr(router_bias), E, top_k, _ptr(partial),
+                                   _ptr(hist), ctypes.byref(ro) if ro is not None else None, _ptr(ws),
+                                   ws.numel() * ws.element_size() if hasattr(ws, "numel") else 0, _stream(stream))
+    return _check(rc, "moe_forward_partial", raise_on_error)
+
+
+def moe_finish_rows(x, total, residual, out, steer=None, stream=None, raise_on_error=True) -> int:
+    """out = bf16((residual ? x : 0) + total), steering projection first when given."""
+    T, H = total.shape
+    rc = lib().moe_finish_rows(_ptr(x), _ptr(total), T, H, int(bool(residual)), _ptr(steer), _ptr(out),
+                               _stream(stream))
+    return _check(rc, "moe_finish_rows", raise_on_error)
 
 
 def moe_route_histogram(expert_offsets, E, L, layer, hist, stream=None, raise_on_error=True) -> int:

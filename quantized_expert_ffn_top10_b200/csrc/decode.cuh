@@ -55,9 +55,11 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 q, float (&v)[8]) {
     v[6] = __uint_as_float(q.w << 16); v[7] = __uint_as_float(q.w & 0xffff0000u);
 }
 
-__device__ __forceinline__ const uint8_t* expert_slot(const DecodeArgs& a, int e, bool& ok) {
+// remote: the slot-table entry is MOE_SLOT_REMOTE (held by another GPU, not an error)
+__device__ __forceinline__ const uint8_t* expert_slot(const DecodeArgs& a, int e, bool& ok, bool& remote) {
     int64_t s = a.slot_table[(int64_t)a.layer * a.E + e];
     ok = (s >= 0 && s < a.n_slots);
+    remote = s == MOE_SLOT_REMOTE;
     return ok ? a.arena + s * a.slot_bytes : nullptr;
 }
 
@@ -73,11 +75,11 @@ __global__ void __launch_bounds__(32 * DEC_GU_WARPS) k_dec_gateup(DecodeArgs a) 
     const int e = a.uniq[blockIdx.y];
     const int r0 = a.offsets[e], n = a.offsets[e + 1] - r0;
     const int H = a.H, I = a.I;
-    bool ok;
-    const uint8_t* slot = expert_slot(a, e, ok);
+    bool ok, remote;
+    const uint8_t* slot = expert_slot(a, e, ok, remote);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (!ok) {  // no valid slot: this expert contributes zero
-        if (threadIdx.x == 0 && blockIdx.x == 0) moe_set_status(MOE_ERR_SLOT);
+        if (threadIdx.x == 0 && blockIdx.x == 0 && !remote) moe_set_status(MOE_ERR_SLOT);
         for (int r = blockIdx.x * 32 + threadIdx.x; r < min(I, (int)(blockIdx.x + 1) * 32); r += blockDim.x)
             for (int j = 0; j < n; ++j) a.h[(size_t)(r0 + j) * I + r] = 0.f;
         return;
@@ -139,8 +141,8 @@ __global__ void __launch_bounds__(32 * DEC_DN_WARPS) k_dec_down(DecodeArgs a) {
     const int e = a.uniq[blockIdx.y];
     const int r0 = a.offsets[e], n = a.offsets[e + 1] - r0;
     const int H = a.H, I = a.I;
-    bool ok;
-    const uint8_t* slot = expert_slot(a, e, ok);
+    bool ok, remote;
+    const uint8_t* slot = expert_slot(a, e, ok, remote);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (!ok) {
         for (int c = blockIdx.x * 32 + threadIdx.x; c < min(H, (int)(blockIdx.x + 1) * 32); c += blockDim.x)
@@ -216,6 +218,30 @@ __global__ void k_combine(const uint16_t* __restrict__ x, const YT* __restrict__
     *reinterpret_cast<uint2*>(out + (size_t)t * H + c) = o;
 }
 
+
+// Partial combine (expert parallelism): part[t][c] = sum_j y[inv[t*k + j]][c]
+// in fp32, j in order, no residual and no rounding.  y is fp32 (decode) or
+// bf16 (prefill); rows of remote experts are zero.
+template <typename YT>
+__global__ void k_combine_f32(const YT* __restrict__ y, const int32_t* __restrict__ inv, int T, int H, int k,
+                              float* __restrict__ part) {
+    const int t = blockIdx.y;
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (t >= T || c >= H) return;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+        const size_t row = (size_t)inv[(size_t)t * k + j] * H + c;
+        if constexpr (sizeof(YT) == 4) {
+            float4 v = __ldg(reinterpret_cast<const float4*>(y + row));
+            acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+        } else {
+            uint2 v = __ldg(reinterpret_cast<const uint2*>(y + row));
+            acc[0] += __uint_as_float(v.x << 16); acc[1] += __uint_as_float(v.x & 0xffff0000u);
+            acc[2] += __uint_as_float(v.y << 16); acc[3] += __uint_as_float(v.y & 0xffff0000u);
+        }
+    }
+    *reinterpret_cast<float4*>(part + (size_t)t * H + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
 
 // Prefill combine for bf16 Y: out[t][c..c+7] = sum_j Y[inv[t][j]][c..c+7] (+ x),
 // summed in j order in fp32; 16-byte loads, four rows in flight.
@@ -313,4 +339,40 @@ __global__ void __launch_bounds__(STEER_THREADS)
     const float dot = s_red[STEER_THREADS / 32];
     for (int c = threadIdx.x; c < H; c += STEER_THREADS)
         out[(size_t)t * H + c] = f32_to_bf16_bits(fmaf(-dot, v[c], s_h[c]));
+}
+
+// The finishing step of an expert-parallel layer: out[t] = bf16(r) with
+// r = (residual ? x[t] : 0) + sum[t] in fp32, projected first when v != NULL
+// (r - (r . v) v, the dot product summed in a fixed order as in
+// k_combine_steer).  One block per token.
+__global__ void __launch_bounds__(STEER_THREADS)
+    k_finish_rows(const uint16_t* __restrict__ x, const float* __restrict__ sum, int T, int H, int residual,
+                  const float* __restrict__ v, uint16_t* __restrict__ out) {
+    extern __shared__ float s_r[];  // [H]
+    __shared__ float s_red[STEER_THREADS / 32 + 1];
+    const int t = blockIdx.x;
+    if (t >= T) return;
+    float part = 0.f;
+    for (int c = threadIdx.x; c < H; c += STEER_THREADS) {
+        const float sv = sum[(size_t)t * H + c];
+        const float r = residual ? sv + bf16_bits_to_f32(x[(size_t)t * H + c]) : sv;
+        s_r[c] = r;
+        if (v) part = fmaf(r, v[c], part);
+    }
+    float dot = 0.f;
+    if (v) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float d = 0.f;
+            for (int w = 0; w < STEER_THREADS / 32; ++w) d += s_red[w];
+            s_red[STEER_THREADS / 32] = d;
+        }
+        __syncthreads();
+        dot = s_red[STEER_THREADS / 32];
+    }
+    for (int c = threadIdx.x; c < H; c += STEER_THREADS)
+        out[(size_t)t * H + c] = f32_to_bf16_bits(v ? fmaf(-dot, v[c], s_r[c]) : s_r[c]);
 }

@@ -1020,7 +1020,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
                     rt.u_e[u] = e;
                     rt.u_pos[u] = r;
                     rt.u_sl[u] = (sl >= 0 && sl < a.n_slots) ? (int32_t)sl : -1;
-                    if (cta == 0 && rt.u_sl[u] < 0) moe_set_status(MOE_ERR_SLOT);
+                    if (cta == 0 && rt.u_sl[u] < 0 && sl != MOE_SLOT_REMOTE) moe_set_status(MOE_ERR_SLOT);
                 }
                 nu += __popc(m);
             }

@@ -344,6 +344,7 @@ struct LayerCall {
     uint8_t* ws;
     size_t ws_bytes;
     cudaStream_t st;
+    float* part;  // expert parallelism: fp32 partial sums instead of out (no residual, no steering)
 };
 
 int check_layer(const LayerCall& c, bool prefill) {
@@ -352,11 +353,14 @@ int check_layer(const LayerCall& c, bool prefill) {
     rc = check_route_args(c.x, c.T, c.d->H, c.W, c.E, c.k, c.ws, prefill ? MOE_PREFILL_MAX_T : MOE_DECODE_MAX_T);
     if (rc) return rc;
     if (c.L < 1 || c.layer < 0 || c.layer >= c.L) return MOE_ERR_RANGE;
-    if (!c.arena || !c.slot_table || !c.out) return MOE_ERR_ARG;
-    if (!aligned(c.arena, 256) || !aligned(c.out, 16) || !aligned(c.steer, 16)) return MOE_ERR_ARG;
-    const size_t xb = (size_t)c.T * c.d->H * 2;
-    const uintptr_t x0 = reinterpret_cast<uintptr_t>(c.x), o0 = reinterpret_cast<uintptr_t>(c.out);
-    if (c.T > 0 && x0 < o0 + xb && o0 < x0 + xb) return MOE_ERR_ARG;
+    if (!c.arena || !c.slot_table || (!c.out && !c.part)) return MOE_ERR_ARG;
+    if (!aligned(c.arena, 256) || !aligned(c.out, 16) || !aligned(c.steer, 16) || !aligned(c.part, 16))
+        return MOE_ERR_ARG;
+    if (c.out) {
+        const size_t xb = (size_t)c.T * c.d->H * 2;
+        const uintptr_t x0 = reinterpret_cast<uintptr_t>(c.x), o0 = reinterpret_cast<uintptr_t>(c.out);
+        if (c.T > 0 && x0 < o0 + xb && o0 < x0 + xb) return MOE_ERR_ARG;
+    }
     if (c.ws_bytes < ws_layout(c.T, c.E, c.k, c.d->H, c.d->I).total) return MOE_ERR_WS;
     return MOE_OK;
 }
@@ -436,11 +440,11 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
     DecodeFusedArgs a{};
     a.arena = c.arena; a.slot_table = c.slot_table; a.n_slots = d->n_slots; a.slot_bytes = d->slot_bytes;
     for (int m = 0; m < 3; ++m) { a.off_codes[m] = d->off_codes[m]; a.off_scales[m] = d->off_scales[m]; }
-    a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.residual;
+    a.H = H; a.I = I; a.E = c.E; a.k = c.k; a.layer = c.layer; a.T = c.T; a.residual = c.part ? 0 : c.residual;
     a.bits_gate = d->bits_gate; a.bits_up = d->bits_up; a.bits_down = d->bits_down;
     a.epc = epc;
     a.x = c.x; a.W = c.W; a.b = c.b; a.out = c.out; a.hist = c.hist;
-    a.hout = c.steer ? reinterpret_cast<float*>(c.ws + L.hout) : nullptr;
+    a.hout = c.part ? c.part : c.steer ? reinterpret_cast<float*>(c.ws + L.hout) : nullptr;
     a.idx = (ro && ro->topk_idx) ? ro->topk_idx : reinterpret_cast<int32_t*>(c.ws + L.idx);
     a.w = (ro && ro->topk_w) ? ro->topk_w : reinterpret_cast<float*>(c.ws + L.w);
     a.offsets = (ro && ro->expert_offsets) ? ro->expert_offsets : reinterpret_cast<int32_t*>(c.ws + L.offsets);
@@ -484,7 +488,7 @@ int run_decode_fused(const LayerCall& c, const DfPlan& plan, int dyn, int epc) {
         case 2408: e = launch_fused<2, 4, 8>(tm, a, grid, dyn, c.st); break;
         default: e = launch_fused<2, 2, 16>(tm, a, grid, dyn, c.st); break;
     }
-    if (e == cudaSuccess && c.steer) {  // steering: the rows leave the kernel in fp32, one block per token finishes them
+    if (e == cudaSuccess && c.steer && !c.part) {  // steering: the rows leave the kernel in fp32, one block per token finishes them
         k_combine_steer<float><<<c.T, STEER_THREADS, H * 4, c.st>>>(nullptr, nullptr, nullptr, a.hout, c.T, H, c.k, 0,
                                                                     c.steer, c.out);
         count(1);
@@ -525,7 +529,10 @@ int run_decode(const LayerCall& c) {
     if (d->bits_down == 4) launch_down<4>(a, umax, c.T, c.st);
     else launch_down<2>(a, umax, c.T, c.st);
     stage(3, c.st);
-    if (c.steer)
+    if (c.part)
+        k_combine_f32<float><<<dim3((d->H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+            a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, d->H, c.k, c.part);
+    else if (c.steer)
         k_combine_steer<float><<<c.T, STEER_THREADS, d->H * 4, c.st>>>(
             c.x, a.y, reinterpret_cast<int32_t*>(c.ws + L.inv), nullptr, c.T, d->H, c.k, c.residual, c.steer, c.out);
     else
@@ -593,7 +600,10 @@ int run_prefill(const LayerCall& c) {
     if (d->bits_down == 4) launch_gemm<1, 4, 4>(th, a, H / PF_BM, mg2, nt, c.st);
     else launch_gemm<1, 2, 2>(th, a, H / PF_BM, mg2, nt, c.st);
     stage(3, c.st);
-    if (c.steer)
+    if (c.part)
+        k_combine_f32<uint16_t><<<dim3((H / 4 + 127) / 128, c.T), 128, 0, c.st>>>(
+            y, reinterpret_cast<int32_t*>(c.ws + L.inv), c.T, H, c.k, c.part);
+    else if (c.steer)
         k_combine_steer<uint16_t><<<c.T, STEER_THREADS, H * 4, c.st>>>(
             c.x, y, reinterpret_cast<int32_t*>(c.ws + L.inv), nullptr, c.T, H, c.k, c.residual, c.steer, c.out);
     else
@@ -702,10 +712,10 @@ int moe_route_static(const uint16_t* x, int T, int H, const float* router_w, con
 static int forward(bool prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L,
                    int layer, const uint16_t* x, int T, const float* router_w, const float* router_bias, int E,
                    int top_k, int residual, const float* steer, uint16_t* out, uint32_t* hist,
-                   const moe_route_out* route_out, void* ws, size_t ws_bytes, void* stream) {
+                   const moe_route_out* route_out, void* ws, size_t ws_bytes, void* stream, float* part = nullptr) {
     LayerCall c{desc, static_cast<const uint8_t*>(arena), slot_table, L, layer, x, T, router_w, router_bias, E,
                 top_k, residual, steer, out, hist, route_out, static_cast<uint8_t*>(ws), ws_bytes,
-                static_cast<cudaStream_t>(stream)};
+                static_cast<cudaStream_t>(stream), part};
     int rc = check_layer(c, prefill);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
@@ -728,6 +738,28 @@ int moe_forward_prefill(const moe_arena_desc* desc, const void* arena, const int
                         void* ws, size_t ws_bytes, void* stream) {
     return forward(true, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, residual, steer, out,
                    hist, route_out, ws, ws_bytes, stream);
+}
+
+int moe_forward_partial(int prefill, const moe_arena_desc* desc, const void* arena, const int32_t* slot_table, int L,
+                        int layer, const uint16_t* x, int T, const float* router_w, const float* router_bias, int E,
+                        int top_k, float* partial, uint32_t* hist, const moe_route_out* route_out, void* ws,
+                        size_t ws_bytes, void* stream) {
+    if (!partial) return MOE_ERR_ARG;
+    return forward(prefill != 0, desc, arena, slot_table, L, layer, x, T, router_w, router_bias, E, top_k, 0, nullptr,
+                   nullptr, hist, route_out, ws, ws_bytes, stream, partial);
+}
+
+int moe_finish_rows(const uint16_t* x, const float* sum, int T, int H, int residual, const float* steer, uint16_t* out,
+                    void* stream) {
+    if (!sum || !out || (residual && !x)) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(sum, 16) || !aligned(steer, 16) || !aligned(out, 16)) return MOE_ERR_ARG;
+    if (T < 0 || H < 8 || H > 8192 || H % 8) return MOE_ERR_SHAPE;
+    if (T == 0) return MOE_OK;
+    const int rc = ensure_init();
+    if (rc) return rc;
+    k_finish_rows<<<T, STEER_THREADS, H * 4, static_cast<cudaStream_t>(stream)>>>(x, sum, T, H, residual, steer, out);
+    count(1);
+    return cuda_rc(cudaGetLastError());
 }
 
 int moe_route_histogram(const int32_t* expert_offsets, int E, int L, int layer, uint32_t* hist, void* stream) {

@@ -199,8 +199,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + C::NACC);
 
     const int64_t slot = a.slot_table[(int64_t)a.layer * a.E + e];
-    if (slot < 0 || slot >= a.n_slots) {  // expert without weights contributes zero
-        if (threadIdx.x == 0) moe_set_status(MOE_ERR_SLOT);
+    if (slot < 0 || slot >= a.n_slots) {  // expert without weights here contributes zero
+        if (threadIdx.x == 0 && slot != MOE_SLOT_REMOTE) moe_set_status(MOE_ERR_SLOT);
         for (int i = threadIdx.x; i < nrows * NOUT; i += blockDim.x)
             a.out[(size_t)(row0 + i / NOUT) * NOUT + i % NOUT] = 0;
         return;

@@ -415,6 +415,13 @@ __device__ __forceinline__ unsigned long long df_key64(double d) {
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
+// The single-warp path with its exact fallback, for a token whose candidates do
+// not certify: rare, so it is a call rather than inlined code in the kernel.
+__device__ __noinline__ void df_topk_fallback(const TopkArgs& a, int t, int32_t* idx_out, float* w_out, int* cs,
+                                              double* cvs, int32_t* nrechk) {
+    topk_token<2>(a, t, idx_out, w_out, cs, cvs, nrechk);
+}
+
 // The selection of topk_token<2> with a shorter first step.  Lanes read the
 // (logit, error bound) records of experts e = lane + 32 i from this CTA's
 // shared-memory copy.  Every entry whose fp32 key is at or above theta, the
@@ -509,7 +516,7 @@ __device__ __forceinline__ void df_topk_token(const TopkArgs& a, const double2* 
     }
     __syncwarp();
     DF_MARK(23);
-    topk_token<2>(a, t, idx_out, w_out, fcs, fcvs, nrechk);
+    df_topk_fallback(a, t, idx_out, w_out, fcs, fcvs, nrechk);
 }
 
 // ---------------------------------------------------------------- phase C: one gate/up unit

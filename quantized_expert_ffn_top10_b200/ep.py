@@ -15,7 +15,7 @@ within rounding, not bit for bit.
 """
 from __future__ import annotations
 
-from . import MOE_DECODE_MAX_T, MOE_SLOT_REMOTE, moe_finish_rows, moe_forward_partial
+from . import MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T, MOE_SLOT_REMOTE, moe_finish_rows, moe_forward_partial
 
 
 def ep_slot_table(slot_table, L: int, E: int, rank: int, G: int):
@@ -55,26 +55,33 @@ def _reduce_rows(partial, T: int, group):
 
 def moe_forward_ep(desc, arena, slot_table_ep, L, layer, x, router_w, router_bias, top_k, residual, out,
                    group=None, prefill=None, steer=None, ws=None, hist=None, stream=None,
-                   partial_fn=None, finish_fn=None):
+                   partial_fn=None, finish_fn=None, max_chunk=MOE_PREFILL_MAX_T):
     """One expert-parallel layer call on this rank's tokens x [T, H] (bf16 as
     int16), writing out [T, H].  slot_table_ep: this rank's table from
-    ep_slot_table.  prefill: the path for the gathered G*T tokens (default: the
-    decode path when they fit it).  partial_fn / finish_fn replace the two
-    library calls (tests on CPU ranks); by default they are moe_forward_partial
-    and moe_finish_rows."""
+    ep_slot_table.  The G*T gathered tokens go through the library in chunks of
+    at most max_chunk rows (one prefill chunk at most); prefill: the path for
+    every chunk (default: the decode path for a chunk that fits it, else the
+    chunk path).  ws must hold the workspace of one chunk.  partial_fn /
+    finish_fn replace the two library calls (tests on CPU ranks) with
+    partial_fn(x_chunk, partial_chunk) and finish_fn(x, total, out); by default
+    they are moe_forward_partial and moe_finish_rows."""
     import torch
     import torch.distributed as dist
+    if not 1 <= max_chunk <= MOE_PREFILL_MAX_T:
+        raise ValueError(f"max_chunk must be in [1, {MOE_PREFILL_MAX_T}], got {max_chunk}")
     G = dist.get_world_size(group)
     T, H = x.shape
     x_all = _gather_rows(x, group)
-    if prefill is None:
-        prefill = G * T > MOE_DECODE_MAX_T
     partial = torch.empty((G * T, H), dtype=torch.float32, device=x.device)
-    if partial_fn is None:
-        moe_forward_partial(prefill, desc, arena, slot_table_ep, L, layer, x_all, router_w, router_bias, top_k,
-                            partial, hist=hist, ws=ws, stream=stream)
-    else:
-        partial_fn(x_all, partial)
+    for c0 in range(0, G * T, max_chunk):  # tokens are independent: any row split gives the same sums
+        c1 = min(G * T, c0 + max_chunk)
+        xc, pc = x_all[c0:c1], partial[c0:c1]
+        if partial_fn is None:
+            pf = (c1 - c0) > MOE_DECODE_MAX_T if prefill is None else prefill
+            moe_forward_partial(pf, desc, arena, slot_table_ep, L, layer, xc, router_w, router_bias, top_k,
+                                pc, hist=hist, ws=ws, stream=stream)
+        else:
+            partial_fn(xc, pc)
     total = _reduce_rows(partial, T, group)
     if finish_fn is None:
         moe_finish_rows(x, total, residual, out, steer=steer, stream=stream)

@@ -4,7 +4,8 @@ rank holds its own tokens, marks the experts it does not hold remote
 oracle stands in for moe_forward_partial, with remote experts as missing
 slots), sums the partials across ranks and finishes its own rows.  The result
 on every rank must be the single-process layer on all tokens: the gather order,
-the owner map and the row slicing of the reduction are what is under test."""
+the owner map, the chunking of the gathered rows and the row slicing of the
+reduction are what is under test."""
 import os
 import socket
 
@@ -26,7 +27,7 @@ def _layer_inputs(G):
     return cfg, cfg.desc(), S.gen_arena_host(cfg), S.gen_slot_table(cfg), S.gen_router(cfg, 0), S.gen_bias(cfg, 0), x
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, max_chunk, out):
     import datetime
     import torch
     import torch.distributed as dist
@@ -42,8 +43,11 @@ def _worker(rank, world, port, out):
         held = set(int(e) for e in range(cfg.E) if tab[e] >= 0)
         assert held == {e for e in range(cfg.E) if e % world == rank}
 
-        def partial_fn(x_all, partial):
-            xb = x_all.numpy().view(np.uint16)
+        chunks = []
+
+        def partial_fn(x_chunk, partial):
+            chunks.append(x_chunk.shape[0])
+            xb = x_chunk.numpy().view(np.uint16)
             miss = np.where(tab < 0, -1, tab).astype(np.int32)  # remote experts: absent here
             ref = O.moe_layer(desc, arena, miss, cfg.L, 0, xb, W, b, cfg.top_k, residual=False)
             partial.copy_(torch.from_numpy(ref["out_f64"].astype(np.float32)))
@@ -55,25 +59,28 @@ def _worker(rank, world, port, out):
         xt = torch.from_numpy(mine.view(np.int16).copy())
         res = torch.zeros((T, cfg.H), dtype=torch.float32)
         moe_forward_ep(desc, None, None, cfg.L, 0, xt, None, None, cfg.top_k, True, res,
-                       partial_fn=partial_fn, finish_fn=finish_fn)
+                       partial_fn=partial_fn, finish_fn=finish_fn, max_chunk=max_chunk)
         out[rank] = res.numpy()
+        out[(rank, "chunks")] = chunks
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_gloo_ranks_reassemble_the_layer(world):
+@pytest.mark.parametrize("world,max_chunk", [(2, 8192), (3, 8192), (3, 5)])
+def test_gloo_ranks_reassemble_the_layer(world, max_chunk):
     import oracle as O
     port = _free_port()
     with mp.Manager() as m:
         out = m.dict()
-        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        mp.spawn(_worker, args=(world, port, max_chunk, out), nprocs=world, join=True)
         res = dict(out)
     cfg, desc, arena, table, W, b, x = _layer_inputs(world)
     ref = O.moe_layer(desc, arena, table, cfg.L, 0, x, W, b, cfg.top_k, residual=True)["out_f64"]
     T = x.shape[0] // world
+    want_chunks = [min(max_chunk, world * T - c) for c in range(0, world * T, max_chunk)]
     for rank in range(world):
+        assert res[(rank, "chunks")] == want_chunks
         got = res[rank]
         want = ref[rank * T:(rank + 1) * T]
         assert got.shape == want.shape

@@ -104,3 +104,44 @@ def test_finish_rows_with_steering_matches_the_steered_layer(cuda_ok):
     torch.cuda.synchronize()
     ref, _ = run_layer(wl, 0, x, prefill=False, residual=True, steer=v)
     assert np.array_equal(out.cpu().numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("case,max_chunk", [("fused_decode", 8192), ("prefill_small", 16)])
+def test_forward_ep_on_one_nccl_rank_is_the_layer(cuda_ok, case, max_chunk):
+    """moe_forward_ep through a one-rank NCCL group: the gather and the
+    reduce-scatter are identities, so the call is the layer (oracle), also when
+    the gathered rows go through the library in several chunks (40 tokens in
+    chunks of 16, 16 and 8: the chunk path twice, then the decode path)."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    import quantized_expert_ffn_top10_b200 as M
+    from quantized_expert_ffn_top10_b200.ep import ep_slot_table, moe_forward_ep
+    if case == "fused_decode":
+        cfg = S.config("decode", seed=99)
+    else:
+        cfg = S.config("tiny", E=16, top_k=4, H=256, I=128, T=40, seed=100)
+    wl = Workload(cfg)
+    x = wl.x_host()
+    T = x.shape[0]
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        table = ep_slot_table(wl.slot_table, cfg.L, cfg.E, 0, 1)
+        xt = torch.from_numpy(x.view(np.int16)).cuda()
+        out = torch.zeros_like(xt)
+        ws = torch.empty(M.moe_workspace_bytes(min(T, max_chunk), cfg.E, cfg.top_k, cfg.H, cfg.I),
+                         dtype=torch.uint8, device="cuda")
+        moe_forward_ep(wl.desc, wl.arena, table, cfg.L, 0, xt, wl.W[0], wl.b[0], cfg.top_k, True, out, ws=ws,
+                       max_chunk=max_chunk)
+        torch.cuda.synchronize()
+        st = M.moe_last_device_error()
+        assert st == 0, f"device status {st}: {M.strerror(st)}"
+    finally:
+        dist.destroy_process_group()
+    ref = wl.oracle_layer(0, x)
+    assert_out_close(out.cpu().numpy().view(np.uint16), ref["out_f64"])

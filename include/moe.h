@@ -59,6 +59,8 @@ extern "C" {
 #define MOE_MAX_E 512         /* experts per layer                              */
 #define MOE_MAX_TOPK 32
 #define MOE_DECODE_MAX_T 8    /* decode path: a verify window of 1 + 4 drafts fits */
+#define MOE_ROUTER_F64_MAX_T 128 /* chunks of up to this many tokens route with fp64
+                                    tensor-core logits; longer ones with bf16 planes */
 #define MOE_PREFILL_MAX_T 8192 /* one prefill chunk                             */
 
 /*
@@ -116,7 +118,11 @@ size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I);
  * "why Coder is fast" (experts addressed and fetched per (layer, expert)):
  * logits l = x W_r^T + b, the top_k experts by (l desc, e asc) - bit-exact
  * against the fp64 sequential definition, certified on the device - their
- * softmax gate weights, and the pairs (t, j) grouped by expert.
+ * softmax gate weights, and the pairs (t, j) grouped by expert.  The logits
+ * that the certification starts from are fp64 with per-entry bounds for
+ * T <= MOE_DECODE_MAX_T, fp64 from the fp64 tensor cores for
+ * T <= MOE_ROUTER_F64_MAX_T, and fp32 sums of exact bf16 planes on the
+ * tensor cores above (E % 128 == 0, H % 64 == 0; other shapes: CUDA cores).
  *   x [T][H] bf16 (device, 16-B aligned), router_w [E][H] fp32 (device,
  *   16-B aligned), router_bias [E] fp32 (device) or NULL.
  *   Outputs (device): topk_idx [T*k], topk_w [T*k], expert_offsets [E+1],
@@ -319,7 +325,7 @@ uint64_t moe_launch_count(void);
  * Both are process-wide and read when a forward call is enqueued.
  * moe_workspace_offset(T, E, top_k, H, I, field): byte offset inside a forward
  *   or route workspace of MOE_WS_FAST_LOGITS (the router's fast logits: fp32
- *   [T][E] for chunks T > MOE_DECODE_MAX_T, fp64 for decode windows) or
+ *   [T][E] for chunks T > MOE_ROUTER_F64_MAX_T, fp64 for shorter ones) or
  *   MOE_WS_PAIR_OUT (per-pair expert outputs w * y in pair order: bf16 [T*k][H]
  *   for chunks) or MOE_WS_SLOW_COUNT (int32: how many tokens of a chunk the
  *   fast certification could not decide, then their ids); (size_t)-1 for bad

@@ -39,7 +39,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 MOE_OK, MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_RANGE = 0, -1, -2, -3
 MOE_ERR_WS, MOE_ERR_CUDA, MOE_ERR_SLOT, MOE_ERR_TIMEOUT = -4, -5, -6, -7
 MOE_ERR_STATIC = -8
-MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T = 8, 8192
+MOE_DECODE_MAX_T, MOE_PREFILL_MAX_T, MOE_ROUTER_F64_MAX_T = 8, 8192, 128
 MOE_ROUTE_STATIC_MAX_T, MOE_ROUTE_STATIC_BYTES = 8, 128 * 1024
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_forward_decode", "moe_forward_prefill",

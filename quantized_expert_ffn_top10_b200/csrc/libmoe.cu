@@ -15,6 +15,7 @@
 #include "perm.cuh"
 #include "prefill.cuh"
 #include "router.cuh"
+#include "router_f64.cuh"
 #include "router_tc.cuh"
 
 namespace {
@@ -33,12 +34,13 @@ Ws ws_layout(int T, int E, int k, int H, int I) {
     const size_t P = (size_t)T * k;
     const size_t nch = (P + PERM_CHUNK - 1) / PERM_CHUNK;
     const bool small = T <= MOE_DECODE_MAX_T;
+    const bool f64r = T <= MOE_ROUTER_F64_MAX_T;  // fp64 router logits (decode windows and short chunks)
     Ws w{};
     size_t o = 0;
     auto put = [&](size_t bytes) { size_t r = o; o += al(std::max<size_t>(bytes, 1)); return r; };
     w.idx = put(P * 4);
     w.w = put(P * 4);
-    w.logit = put((size_t)T * E * (small ? 8 : 4));  // fp64 logits for decode windows, fp32 for chunks
+    w.logit = put((size_t)T * E * (f64r ? 8 : 4));  // fp64 logits up to MOE_ROUTER_F64_MAX_T, fp32 above
     w.absum = put(small ? (size_t)T * E * 8 : 0);
     w.cmax = put((size_t)E * 4);                    // router row norms
     w.offsets = put((size_t)(E + 1) * 4);
@@ -145,6 +147,13 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
         ta.absum = absum;
         ta.gfast = gamma_n(H / 32 + 6, 1.1102230246251565e-16);
         k_topk<1><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
+    } else if (T <= MOE_ROUTER_F64_MAX_T) {  // short chunk: fp64 tensor-core logits, bound from norms
+        double* logit = reinterpret_cast<double*>(ws + L.logit);
+        float* wnorm = reinterpret_cast<float*>(ws + L.cmax);
+        k_router_f64<<<dim3((E + 7) / 8, (T + 7) / 8), 32 * RF_WARPS, 0, st>>>(x, T, H, W, b, E, logit, wnorm);
+        ta.wnorm = wnorm;
+        ta.gfast = (double)(H + 32) * 1.1102230246251565e-16 * 1.01;
+        k_topk<2><<<tk_grid, 32 * MOE_TOPK_WARPS, 0, st>>>(ta);
     } else {
         float* wnorm = reinterpret_cast<float*>(ws + L.cmax);
         float* logit = reinterpret_cast<float*>(ws + L.logit);
@@ -194,7 +203,7 @@ int launch_route(const uint16_t* x, int T, int H, const float* W, const float* b
     k_perm_count<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
     k_perm_scan<<<1, MOE_MAX_E, 0, st>>>(pa);
     k_perm_scatter<<<pa.nchunks, PERM_CHUNK, 0, st>>>(pa);
-    count(T <= MOE_DECODE_MAX_T ? 5 : 9);
+    count(T <= MOE_ROUTER_F64_MAX_T ? 5 : 9);
     return cuda_rc(cudaGetLastError());
 }
 
@@ -907,6 +916,7 @@ size_t moe_workspace_offset(int T, int E, int top_k, int H, int I, int field) {
 
 double moe_router_gamma(int T, int E, int H) {
     if (T <= MOE_DECODE_MAX_T || E < 1 || E > MOE_MAX_E || H < 32 || H % 32) return -1.0;
+    if (T <= MOE_ROUTER_F64_MAX_T) return (double)(H + 32) * 1.1102230246251565e-16 * 1.01;  // fp64 tensor cores
     if (E % RT_BM == 0 && H % RT_BK == 0) return moe_tc_router_gamma(H);  // tensor-core chunk router
     return gamma_n(RG_BK + H / RG_BK + 2, 5.9604644775390625e-8);      // CUDA-core chunk router
 }

@@ -30,6 +30,22 @@ def test_every_declared_function_is_exported(lib):
         assert hasattr(so, n), n
 
 
+def test_binding_constants_match_the_header():
+    """Every integer #define MOE_* of the header has the same value in the
+    binding (the ones the binding names)."""
+    hdr = open(B.sources()[-1]).read()
+    defs = {n: int(v.strip("()").replace(" ", "").split("*")[0]) * (
+        int(v.strip("()").replace(" ", "").split("*")[1]) if "*" in v else 1)
+        for n, v in re.findall(r"^#define\s+(MOE_\w+)\s+(\(?-?\d+(?:\s*\*\s*\d+)?\)?)", hdr, re.M)}
+    assert {"MOE_DECODE_MAX_T", "MOE_ROUTER_F64_MAX_T", "MOE_SLOT_REMOTE", "MOE_ERR_TIMEOUT"} <= set(defs)
+    checked = 0
+    for n, v in defs.items():
+        if hasattr(M, n):
+            assert getattr(M, n) == v, n
+            checked += 1
+    assert checked >= 10
+
+
 def test_workspace_bytes_grows_with_T(lib):
     a = M.moe_workspace_bytes(5, 512, 10, 2048, 512)
     b = M.moe_workspace_bytes(8192, 512, 10, 2048, 512)

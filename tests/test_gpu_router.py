@@ -1,7 +1,8 @@
-"""The chunk router (tensor-core logits + certified top-k, taken by every call
-with T > 8, E % 128 == 0 and H % 64 == 0) on exact ties, near ties, a zero
-token and a huge-norm token; the measured slack of its error bound on the
-full-size workloads; and moe_route_histogram through the C ABI."""
+"""The chunk routers - fp64 tensor-core logits for 8 < T <= 128, bf16-plane
+tensor-core logits above (E % 128 == 0 and H % 64 == 0), each with a certified
+top-k - on exact ties, near ties, a zero token and a huge-norm token; the
+measured slack of their error bounds; and moe_route_histogram through the C
+ABI."""
 import numpy as np
 import pytest
 
@@ -13,7 +14,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _route(x_bits, W, b, k, want_logits=False):
-    """moe_route on host inputs; returns the routing (and the fast logits)."""
+    """moe_route on host inputs; returns the routing (and the fast logits:
+    fp64 up to MOE_ROUTER_F64_MAX_T tokens, fp32 above)."""
     import torch
     import quantized_expert_ffn_top10_b200 as M
     T, H = x_bits.shape
@@ -31,7 +33,9 @@ def _route(x_bits, W, b, k, want_logits=False):
     res["topk_w"] = res["topk_w"].reshape(T, k)
     if want_logits:
         off = M.moe_workspace_offset(T, E, k, H, 32, M.MOE_WS_FAST_LOGITS)
-        res["fast"] = ws[off:off + T * E * 4].view(torch.float32).reshape(T, E).cpu().numpy()
+        f64 = T <= M.MOE_ROUTER_F64_MAX_T
+        nb = T * E * (8 if f64 else 4)
+        res["fast"] = ws[off:off + nb].view(torch.float64 if f64 else torch.float32).reshape(T, E).cpu().numpy()
     return res
 
 
@@ -44,10 +48,10 @@ def _ranks(x_bits, W, b):
     return lg
 
 
-def _tie_workload():
-    """E = 512, H = 2048, T = 256: rows edited so that exact ties and 1-ulp near
-    ties fall inside chosen tokens' top 10 and on their 10th / 11th boundary."""
-    cfg = S.config("prefill", T=256, seed=31)
+def _tie_workload(T=256):
+    """E = 512, H = 2048: rows edited so that exact ties and 1-ulp near ties
+    fall inside chosen tokens' top 10 and on their 10th / 11th boundary."""
+    cfg = S.config("prefill", T=T, seed=31)
     x = S.gen_x(cfg)
     W = S.gen_router(cfg)
     W[:8] *= 3.0                                   # hot rows: in most tokens' top 10
@@ -78,8 +82,9 @@ def _tie_workload():
     return cfg, x, W, boundary
 
 
-def test_chunk_router_exact_and_near_ties(cuda_ok):
-    cfg, x, W, boundary = _tie_workload()
+@pytest.mark.parametrize("T", [64, 256])  # fp64 tensor-core router; bf16-plane tensor-core router
+def test_chunk_router_exact_and_near_ties(cuda_ok, T):
+    cfg, x, W, boundary = _tie_workload(T)
     k, E = cfg.top_k, cfg.E
     assert len(boundary) >= 6
     res = _route(x, W, None, k)
@@ -98,11 +103,12 @@ def test_chunk_router_exact_and_near_ties(cuda_ok):
         assert (e10 in idx[t]) == (e10 in res["topk_idx"][t]) and (e11 in idx[t]) == (e11 in res["topk_idx"][t])
 
 
-def test_chunk_router_ties_through_the_layer(cuda_ok):
-    """The same edited router in a full prefill call: routing of all 256
-    tokens, outputs of the edited tokens and a sample."""
+@pytest.mark.parametrize("T", [64, 256])
+def test_chunk_router_ties_through_the_layer(cuda_ok, T):
+    """The same edited router in a full prefill call: routing of all tokens,
+    outputs of the edited tokens and a sample."""
     import torch
-    cfg, x, W, boundary = _tie_workload()
+    cfg, x, W, boundary = _tie_workload(T)
     wl = Workload(cfg, device_arena=True)
     wl.W_host[0] = W
     wl.W[0] = torch.from_numpy(W).cuda()
@@ -110,7 +116,7 @@ def test_chunk_router_ties_through_the_layer(cuda_ok):
     lg = O.router_logits(x, W, None)
     idx, w = O.topk(lg, cfg.top_k)
     check_routing(res, idx, w, cfg.E)
-    toks = sorted({0, 1, *[t for t, _, _ in boundary], 100, 200, 255})
+    toks = sorted(t for t in {0, 1, *[t for t, _, _ in boundary], 50, 100, 200, T - 1} if t < T)
     ref = wl.oracle_layer(0, x, tokens=np.array(toks, np.int32))
     assert_out_close(out, ref["out_f64"], rows=toks)
 
@@ -139,6 +145,33 @@ def test_chunk_router_bound_slack(cuda_ok, name, layer):
     ulps = float((err / (2.0 ** -23 * (np.abs(xf) @ np.abs(Wf).T + babs[None, :]))).max())
     print(f"\n[router bound slack] {name}: max |fast - exact| / bound = {ratio:.4f}; "
           f"max error = {ulps:.3f} x 2^-23 sum|x w|; gamma = {gamma:.3e}")
+    assert ratio < 1.0
+    idx, w = O.topk(exact, cfg.top_k)
+    check_routing(res, idx, w, cfg.E)
+
+
+@pytest.mark.parametrize("name,layer,T", [("prefill", 0, 128), ("prefill_stack", 5, 100)])
+def test_short_chunk_router_bound_slack(cuda_ok, name, layer, T):
+    """The fp64 tensor-core logits of short chunks against the fp64 definition:
+    |fast - exact| <= gamma (||x_t|| ||W_r[e]|| + |b_e|) for every (token,
+    expert), gamma = moe_router_gamma's gamma_(H+32); the ratio is printed as
+    the measured slack.  The routing is the definition's."""
+    import quantized_expert_ffn_top10_b200 as M
+    cfg = S.config(name, T=T)
+    x = S.gen_x(cfg)
+    W = S.gen_router(cfg, layer)
+    b = S.gen_bias(cfg, layer)
+    res = _route(x, W, b, cfg.top_k, want_logits=True)
+    exact = O.router_logits(x, W, b)
+    gamma = M.moe_router_gamma(T, cfg.E, cfg.H)
+    assert 0 < gamma < 1e-12
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    Wf = W.astype(np.float64)
+    babs = np.zeros(cfg.E) if b is None else np.abs(b.astype(np.float64))
+    bound = gamma * (np.linalg.norm(xf, axis=1)[:, None] * np.linalg.norm(Wf, axis=1)[None, :] + babs[None, :])
+    err = np.abs(res["fast"] - exact)
+    ratio = float((err / bound).max())
+    print(f"\n[short-chunk router bound slack] {name}: max |fast - exact| / bound = {ratio:.2e}; gamma = {gamma:.3e}")
     assert ratio < 1.0
     idx, w = O.topk(exact, cfg.top_k)
     check_routing(res, idx, w, cfg.E)

@@ -2,7 +2,8 @@
 the router is replicated, and one exchange step surrounds the layer:
 
     x      [T, H] bf16 per GPU  --all-gather-->  [G*T, H] on every GPU
-    moe_forward_partial on the gathered tokens, remote experts contributing 0
+    moe_forward_partial on the gathered tokens (in chunks of at most one
+        prefill chunk), remote experts contributing 0
     partial [G*T, H] fp32       --reduce-scatter (sum)-->  [T, H] per GPU
     moe_finish_rows: residual, steering, one bf16 rounding
 

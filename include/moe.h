@@ -108,7 +108,9 @@ typedef struct moe_route_out {
 } moe_route_out;
 
 /* Bytes of scratch workspace a forward (or moe_route) call with these sizes
- * needs; pass it as `ws` (device, 256-byte aligned).  Host only, no CUDA. */
+ * needs; pass it as `ws` (device, 256-byte aligned).  Non-decreasing in T: a
+ * workspace sized for T serves every call with at most T tokens and the same
+ * E, top_k, H and I.  Host only, no CUDA. */
 size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I);
 
 /*

@@ -631,7 +631,12 @@ extern "C" {
 
 size_t moe_workspace_bytes(int T, int E, int top_k, int H, int I) {
     if (T < 0 || E < 1 || top_k < 1 || H < 1 || I < 1) return 0;
-    return ws_layout(T, E, top_k, H, I).total;
+    // the layout grows with T inside each router regime; across a regime's upper
+    // limit it can shrink, so the size is the largest over every T' <= T
+    size_t b = ws_layout(T, E, top_k, H, I).total;
+    for (const int lim : {MOE_DECODE_MAX_T, MOE_ROUTER_F64_MAX_T})
+        if (T > lim) b = std::max(b, ws_layout(lim, E, top_k, H, I).total);
+    return b;
 }
 
 int moe_route(const uint16_t* x, int T, int H, const float* router_w, const float* router_bias, int E, int top_k,

@@ -53,6 +53,18 @@ def test_workspace_bytes_grows_with_T(lib):
     assert M.moe_workspace_bytes(-1, 512, 10, 2048, 512) == 0
 
 
+@pytest.mark.parametrize("shape", [(512, 10, 2048, 512), (256, 10, 2048, 512), (16, 4, 256, 128), (8, 2, 64, 32)])
+def test_workspace_bytes_never_shrinks_with_T(lib, shape):
+    """A workspace sized for T serves every shorter call: the size is
+    non-decreasing in T, also across the router regimes' limits (8 and 128
+    tokens, where the layout itself shrinks)."""
+    E, k, H, I = shape
+    Ts = list(range(0, 300)) + [511, 512, 4095, 4096, 8191, 8192]
+    sizes = [M.moe_workspace_bytes(T, E, k, H, I) for T in Ts]
+    assert all(b >= a for a, b in zip(sizes, sizes[1:]))
+    assert all(b % 256 == 0 for b in sizes)
+
+
 def _fwd(fn, desc, T=5, E=512, k=10, L=1, layer=0, x=FAKE, out=FAKE + (1 << 16), ws=FAKE * 64,
          ws_bytes=None, arena=FAKE * 128, W=FAKE * 4, steer=None):
     d = M.as_desc(desc) if desc is not None else None

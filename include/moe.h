@@ -240,7 +240,9 @@ int moe_forward_partial(int prefill, const moe_arena_desc* desc, const void* are
  * with the steering projection applied first when steer != NULL (as in the
  * forwards: r - (r . v) v on the fp32 row, residual included).  x [T][H] bf16,
  * sum [T][H] fp32, steer [H] fp32 or NULL, out [T][H] bf16, all device,
- * 16-B aligned; H % 8 == 0.  The finishing step of an expert-parallel layer.
+ * 16-B aligned; H % 8 == 0.  The finishing step of an expert-parallel layer
+ * (the combine's last two steps of the "Coder benchmark record" page's layer:
+ * residual add and one rounding; steering as its steering vector section).
  */
 int moe_finish_rows(const uint16_t* x, const float* sum, int T, int H, int residual, const float* steer,
                     uint16_t* out, void* stream);
@@ -292,10 +294,13 @@ double moe_profile_hit_rate(const uint16_t* pairs, int n_pairs, int L, int E, in
 /* Reads and clears the current device's status word after synchronising
  * `stream`: MOE_OK, MOE_ERR_SLOT or MOE_ERR_TIMEOUT (the first latched), or
  * MOE_ERR_RANGE if an internal index was out of range and replaced (a
- * library fault; inputs cannot cause it: non-finite logits rank as -inf). */
+ * library fault; inputs cannot cause it: non-finite logits rank as -inf).
+ * No page defines it: it is the boundary's way of reporting what the device
+ * detects without trapping. */
 int moe_last_device_error(void* stream);
 
-/* Static message for a return code. */
+/* Static message for a return code (the boundary's error contract; no page
+ * defines it).  Never NULL: an unknown code gets a generic message. */
 const char* moe_strerror(int code);
 
 /*

@@ -131,3 +131,21 @@ def test_mid_T_distinct_experts(T, lo, hi):
     cnt, _ = _routing_counts(S.gen_x(cfg), S.gen_router(cfg), None, cfg.top_k)
     nz = cnt[cnt > 0]
     assert lo <= nz.size <= hi and nz.max() <= 14
+
+
+def test_pruned_stack_traffic_is_concentrated():
+    """The 48 x 256 stack under its Zipf bias, 20 windows of 5 tokens per
+    layer: the 300 most routed of the 12,288 (layer, expert) pairs take about
+    half of the routed reads (48% in this draw) and the first 2,537 nearly all
+    (98%): a few hundred experts carry much of the traffic."""
+    cfg = S.config("decode_stack")
+    tot = np.zeros((cfg.L, cfg.E))
+    for layer in range(cfg.L):
+        W, b = S.gen_router(cfg, layer), S.gen_bias(cfg, layer)
+        x = np.concatenate([S.gen_x(cfg, 5, stream_offset=o) for o in range(20)])
+        cnt, _ = _routing_counts(x, W, b, cfg.top_k)
+        tot[layer] = cnt
+    f = np.sort(tot.ravel())[::-1]
+    assert f.sum() == cfg.L * 20 * 5 * cfg.top_k
+    assert 0.40 < f[:300].sum() / f.sum() < 0.56
+    assert f[:2537].sum() / f.sum() > 0.95

@@ -150,3 +150,11 @@ def test_route_static_checks(lib):
     assert lib.moe_route_static(FAKE + 2, 5, 2048, FAKE, None, 512, 10, FAKE, FAKE, FAKE, FAKE, None) \
         == M.MOE_ERR_ARG
     assert lib.moe_route_static(FAKE, 0, 2048, FAKE, None, 512, 10, FAKE, FAKE, FAKE, FAKE, None) == M.MOE_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libmoe.so the binding raises; there is no CPU fallback."""
+    monkeypatch.setattr(M, "_lib", None)
+    monkeypatch.setattr(M, "LIB_PATH", str(tmp_path / "libmoe.so"))
+    with pytest.raises(ImportError):
+        M.moe_workspace_bytes(5, 512, 10, 2048, 512)

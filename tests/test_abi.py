@@ -158,3 +158,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(M, "LIB_PATH", str(tmp_path / "libmoe.so"))
     with pytest.raises(ImportError):
         M.moe_workspace_bytes(5, 512, 10, 2048, 512)
+
+
+@pytest.mark.parametrize("T", [1, 5, 8, 9, 64, 128, 129, 300, 8192])
+def test_workspace_fields_are_aligned_and_inside(lib, T):
+    """The workspace fields the tests read sit on 256-byte boundaries inside
+    the workspace, and the fast logits' region holds T x E values of the
+    router's dtype (fp64 up to MOE_ROUTER_F64_MAX_T tokens, fp32 above)."""
+    E, k, H, I = 512, 10, 2048, 512
+    total = M.moe_workspace_bytes(T, E, k, H, I)
+    offs = {f: M.moe_workspace_offset(T, E, k, H, I, f)
+            for f in (M.MOE_WS_FAST_LOGITS, M.MOE_WS_PAIR_OUT, M.MOE_WS_SLOW_COUNT)}
+    for f, o in offs.items():
+        assert o % 256 == 0 and o < total, (f, o, total)
+    nb = T * E * (8 if T <= M.MOE_ROUTER_F64_MAX_T else 4)
+    later = [o for o in offs.values() if o > offs[M.MOE_WS_FAST_LOGITS]]
+    assert offs[M.MOE_WS_FAST_LOGITS] + nb <= min(later + [total])
+    with pytest.raises(M.MoeError):
+        M.moe_workspace_offset(T, E, k, H, I, 99)  # unknown field
